@@ -1,0 +1,212 @@
+"""CPU oracle for the NVFP4 routed-expert MoE layer.
+
+TEST INFRASTRUCTURE ONLY.  The oracle is the slow, plain statement of what the CUDA
+library computes; it proves the library's results.  Only the test suite,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import it.
+The product path (``bit_quantized_moe_nvfp4_b200``) never imports, links or runs it,
+and the two share no code: they meet only on the seeded inputs made by ``synth``.
+
+The arithmetic lives in ``nvfp4_oracle.c`` (plain C, fp32 codec steps, fp64 MoE
+accumulation); this module compiles it with gcc on first use and marshals numpy arrays
+through ctypes.  Sources followed: page "GLM-5-NVFP4-MTP", sections "Model
+Description" (NVFP4: 4-bit values, one FP8 scale per 16 elements; 256 experts, top-8)
+and "What's quantized" (routed-expert gate/up/down projections only).
+
+Pins (tests/test_oracle.py): the exhaustive E2M1 table, every E4M3 code against
+torch's float8_e4m3fn, a hand-worked block, quantizer invariants, the routing
+permutation against a stable sort, and the MoE against a dense brute force.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+# gcc flags: IEEE fp32/fp64 with no contraction into FMA and no fast-math, so every
+# operation rounds exactly as the C source states.
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+          "-fno-fast-math", "-Wall"]
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to the C source (gcc).  Returns its path."""
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64 = ctypes.c_int64
+            L.oracle_e2m1_value.restype = ctypes.c_double
+            L.oracle_e2m1_value.argtypes = [ctypes.c_int]
+            L.oracle_e4m3_value.restype = ctypes.c_double
+            L.oracle_e4m3_value.argtypes = [ctypes.c_int]
+            L.oracle_e2m1_encode.restype = ctypes.c_int
+            L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+            L.oracle_e4m3_encode.restype = ctypes.c_int
+            L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            L.oracle_bf16_round.restype = ctypes.c_uint16
+            L.oracle_bf16_round.argtypes = [ctypes.c_double]
+            L.oracle_global_scale.restype = ctypes.c_float
+            L.oracle_global_scale.argtypes = [P, I64]
+            L.oracle_nvfp4_quantize.restype = None
+            L.oracle_nvfp4_quantize.argtypes = [P, I64, I64, I64, P, P, P]
+            L.oracle_nvfp4_dequantize.restype = None
+            L.oracle_nvfp4_dequantize.argtypes = [P, P, P, I64, I64, I64, P]
+            L.oracle_route.restype = I64
+            L.oracle_route.argtypes = [P, I64, I64, I64, P, P, P, P]
+            L.oracle_moe_forward.restype = I64
+            L.oracle_moe_forward.argtypes = [P, P, P, I64, I64, I64, I64, I64,
+                                             P, P, P, P, P, P, P, I64, P, P]
+            L.oracle_threads.restype = ctypes.c_int
+            L.oracle_threads.argtypes = []
+            L.oracle_set_threads.restype = None
+            L.oracle_set_threads.argtypes = [ctypes.c_int]
+            _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    """bf16 data as a C-contiguous uint16 numpy array (accepts torch bf16 tensors)."""
+    if hasattr(a, "detach"):
+        import torch
+        a = a.detach().to("cpu").contiguous().view(torch.int16).numpy()
+    return np.ascontiguousarray(a).view(np.uint16)
+
+
+def _np(a, dtype) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").contiguous().numpy()
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ----------------------------------------------------------------------------- formats
+def e2m1_value(code: int) -> float:
+    return _load().oracle_e2m1_value(int(code))
+
+
+def e4m3_value(code: int) -> float:
+    return _load().oracle_e4m3_value(int(code))
+
+
+def e2m1_encode(v: float) -> int:
+    return _load().oracle_e2m1_encode(float(v))
+
+
+def e4m3_encode(v: float) -> int:
+    return _load().oracle_e4m3_encode(float(v))
+
+
+def bf16_round(v: float) -> int:
+    """bf16 bits of the nearest bf16 to v (one rounding from the fp64 value)."""
+    return int(_load().oracle_bf16_round(float(v)))
+
+
+def threads() -> int:
+    return int(_load().oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+# ----------------------------------------------------------------------------- codec
+def global_scale(x) -> float:
+    xs = _u16(x).reshape(-1)
+    return float(_load().oracle_global_scale(_p(xs), xs.size))
+
+
+def quantize(x):
+    """x: bf16 [n, rows, cols] (or [rows, cols]) -> (packed u8 [n,rows,cols/2],
+    scales u8 [n,rows,cols/16], g fp32 [n])."""
+    xs = _u16(x)
+    if xs.ndim == 2:
+        xs = xs[None]
+    n, rows, cols = xs.shape
+    assert cols % 16 == 0
+    packed = np.zeros((n, rows, cols // 2), np.uint8)
+    scales = np.zeros((n, rows, cols // 16), np.uint8)
+    g = np.zeros((n,), np.float32)
+    _load().oracle_nvfp4_quantize(_p(xs), n, rows, cols, _p(packed), _p(scales), _p(g))
+    return packed, scales, g
+
+
+def dequantize(packed, scales, g):
+    """-> bf16 bits as uint16 [n, rows, cols]."""
+    pk = _np(packed, np.uint8)
+    sc = _np(scales, np.uint8)
+    gs = _np(g, np.float32).reshape(-1)
+    if pk.ndim == 2:
+        pk, sc = pk[None], sc[None]
+    n, rows, half = pk.shape
+    cols = half * 2
+    out = np.zeros((n, rows, cols), np.uint16)
+    _load().oracle_nvfp4_dequantize(_p(pk), _p(sc), _p(gs), n, rows, cols, _p(out))
+    return out
+
+
+# ----------------------------------------------------------------------------- routing
+def route(ids, E: int):
+    """ids int32 [T, K] -> (counts [E], offsets [E+1], perm [n_valid], inv [T*K], n_bad)."""
+    a = _np(ids, np.int32)
+    T, K = a.shape
+    counts = np.zeros((E,), np.int32)
+    offsets = np.zeros((E + 1,), np.int32)
+    perm = np.zeros((T * K,), np.int32)
+    inv = np.zeros((T * K,), np.int32)
+    bad = _load().oracle_route(_p(a), T, K, E, _p(counts), _p(offsets), _p(perm), _p(inv))
+    return counts, offsets, perm[: offsets[E]], inv, int(bad)
+
+
+# ----------------------------------------------------------------------------- MoE
+def moe_forward(x, ids, w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, tokens=None):
+    """Routed-expert MoE forward for the listed tokens (all when tokens is None).
+
+    x bf16 [T,H]; ids int32 [T,K]; w fp32 [T,K]; w_gu u8 [E,2I,H/2]; s_gu u8 [E,2I,H/16];
+    g_gu fp32 [E]; w_dn u8 [E,H,I/2]; s_dn u8 [E,H,I/16]; g_dn fp32 [E].
+    Returns (out bf16 bits uint16 [n,H], out fp64 [n,H], number of out-of-range ids).
+    """
+    xs = _u16(x)
+    T, H = xs.shape
+    ia = _np(ids, np.int32)
+    wa = _np(w, np.float32)
+    K = ia.shape[1]
+    pg, sg, gg = _np(w_gu, np.uint8), _np(s_gu, np.uint8), _np(g_gu, np.float32)
+    pd, sd, gd = _np(w_dn, np.uint8), _np(s_dn, np.uint8), _np(g_dn, np.float32)
+    E = pg.shape[0]
+    I = pg.shape[1] // 2
+    assert pg.shape == (E, 2 * I, H // 2) and sg.shape == (E, 2 * I, H // 16)
+    assert pd.shape == (E, H, I // 2) and sd.shape == (E, H, I // 16)
+    tok = np.arange(T, dtype=np.int64) if tokens is None else _np(tokens, np.int64)
+    out = np.zeros((tok.size, H), np.uint16)
+    out64 = np.zeros((tok.size, H), np.float64)
+    bad = _load().oracle_moe_forward(_p(xs), _p(ia), _p(wa), T, H, I, E, K,
+                                     _p(pg), _p(sg), _p(gg), _p(pd), _p(sd), _p(gd),
+                                     _p(tok), tok.size, _p(out), _p(out64))
+    return out, out64, int(bad)
+
+
+def bf16_bits_to_f32(u16: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to fp32 (exact)."""
+    return (np.asarray(u16, np.uint16).astype(np.uint32) << 16).view(np.float32)

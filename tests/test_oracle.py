@@ -1,0 +1,286 @@
+"""Pins for the CPU oracle: it is checked against what the format definitions, the
+mathematics and independent library routines fix, never against itself.
+
+Format sources: page "GLM-5-NVFP4-MTP", "Model Description" (NVFP4 = 4-bit values with
+one FP8 scale per 16 elements; 256 experts, 8 active) and "What's quantized" (routed
+expert gate/up/down only).  E2M1 elements, E4M3 scales, one fp32 global scale per tensor
+and block scale = amax/6 rounded to E4M3 complete the definition.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+# E2M1 codes 0..15 by the bit-field definition (sign | 2-bit exponent, bias 1 | 1-bit
+# mantissa; exponent 0 is subnormal), written out value by value.
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,
+              -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def e4m3_torch(codes):
+    """E4M3 values through torch's float8_e4m3fn (an independent decoder)."""
+    c = torch.as_tensor(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return c.to(torch.float64).numpy()
+
+
+# ------------------------------------------------------------------------------ E2M1
+def test_e2m1_table_exhaustive():
+    for code, want in enumerate(E2M1_TABLE):
+        got = oracle.e2m1_value(code)
+        assert got == want and np.signbit(got) == np.signbit(want), (code, got, want)
+
+
+@pytest.mark.parametrize("v,code", [
+    (0.0, 0x0), (-0.0, 0x8), (0.1, 0x0), (-0.1, 0x8),
+    (0.25, 0x0), (0.2500001, 0x1), (0.75, 0x2), (0.7499999, 0x1),
+    (1.25, 0x2), (1.2500001, 0x3), (1.75, 0x4), (2.5, 0x4), (2.5000002, 0x5),
+    (3.5, 0x6), (3.4999998, 0x5), (5.0, 0x6), (5.0000005, 0x7), (6.0, 0x7),
+    (6.5, 0x7), (1e30, 0x7), (-1e30, 0xF), (-2.75, 0xD), (-0.3, 0x9), (4.9, 0x6),
+])
+def test_e2m1_encode_ties_and_saturation(v, code):
+    # Ties go to the even code (mantissa bit 0); above 6 saturates; sign kept on zero.
+    assert oracle.e2m1_encode(v) == code
+
+
+def test_e2m1_encode_roundtrip_every_code():
+    for code, val in enumerate(E2M1_TABLE):
+        assert oracle.e2m1_encode(val) == code
+
+
+# ------------------------------------------------------------------------------ E4M3
+def test_e4m3_every_code_matches_torch_float8():
+    ref = e4m3_torch(np.arange(256))
+    for code in range(256):
+        got = oracle.e4m3_value(code)
+        if np.isnan(ref[code]):
+            assert np.isnan(got) and (code & 0x7F) == 0x7F
+        else:
+            assert got == ref[code], (code, got, ref[code])
+
+
+def test_e4m3_spot_values():
+    assert oracle.e4m3_value(0x7E) == 448.0          # largest finite
+    assert oracle.e4m3_value(0x08) == 2.0 ** -6      # smallest normal
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9      # smallest subnormal
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9  # largest subnormal
+    assert oracle.e4m3_value(0x38) == 1.0
+    assert oracle.e4m3_value(0x55) == 13.0
+
+
+def test_e4m3_monotone_and_roundtrip():
+    vals = [oracle.e4m3_value(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))
+    for c in range(0x7F):
+        assert oracle.e4m3_encode(vals[c]) == c
+
+
+def test_e4m3_encode_matches_torch_rne():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([
+        rng.uniform(0, 464, 4000), np.exp(rng.uniform(np.log(1e-4), np.log(448), 4000)),
+        rng.uniform(0, 2.0 ** -6, 1000)]).astype(np.float32)
+    # midpoints between neighbouring codes: ties to even
+    vals = np.array([oracle.e4m3_value(c) for c in range(0x7F)])
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    v = np.concatenate([v, mids, np.float32(448.0) + np.float32(15.9)[None]])
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(x) for x in v], np.uint8)
+    assert np.array_equal(got, want)
+
+
+def test_e4m3_saturates_instead_of_nan():
+    for v in (448.0, 463.9, 464.0, 500.0, 1e6, 3e38):
+        assert oracle.e4m3_encode(v) == 0x7E
+
+
+# ------------------------------------------------------------------------------ bf16
+def test_bf16_round_matches_torch_from_fp32():
+    rng = np.random.default_rng(2)
+    v = np.concatenate([rng.standard_normal(20000) * 10 ** rng.uniform(-30, 30, 20000),
+                        [0.0, -0.0, 1.0, -3.0]]).astype(np.float32)
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.bf16_round(float(x)) for x in v], np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_bf16_round_is_single_rounding_from_fp64():
+    # 1 + 2^-8 is the midpoint between bf16 1.0 and 1 + 2^-7.  A value just above it
+    # must round up; rounding through fp32 first would land on the midpoint and go even.
+    assert oracle.bf16_round(1.0 + 2.0 ** -8 + 2.0 ** -30) == 0x3F81
+    assert oracle.bf16_round(1.0 + 2.0 ** -8) == 0x3F80            # tie -> even
+    assert oracle.bf16_round(1.0 + 3 * 2.0 ** -8) == 0x3F82        # tie -> even (up)
+
+
+# ------------------------------------------------------------------------------ codec
+def _bf16_bits(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16)
+
+
+def test_hand_worked_blocks():
+    """Two 16-element blocks worked by hand (tests/golden/hand_block.json)."""
+    with open(os.path.join(GOLDEN, "hand_block.json")) as f:
+        gold = json.load(f)
+    x = _bf16_bits(gold["x"]).reshape(1, 1, 32)
+    assert torch.equal(x.float().reshape(-1), torch.tensor(gold["x"]))  # exact in bf16
+    packed, scales, g = oracle.quantize(x)
+    assert g[0] == np.float32(gold["g"])
+    assert list(scales.reshape(-1)) == gold["scales"]
+    assert list(packed.reshape(-1)) == [int(b, 16) for b in gold["packed_hex"]]
+    deq = oracle.dequantize(packed, scales, g)
+    want = _bf16_bits(gold["dequant"]).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(deq.reshape(-1), want)
+
+
+def _decode_with_tables(packed, scales, g):
+    """fp64 weights from packed codes, using the written-out E2M1 table and torch's E4M3."""
+    lo = packed & 0xF
+    hi = packed >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(*packed.shape[:-1], packed.shape[-1] * 2)
+    q = np.asarray(E2M1_TABLE)[codes]
+    s = np.repeat(e4m3_torch(scales), 16, axis=-1)
+    return q * s * np.asarray(g, np.float64).reshape(-1, *([1] * (packed.ndim - 1)))
+
+
+def test_quantize_invariants_random():
+    x = synth.normal_bf16((3, 24, 96), 7, "inv", std=0.02, outlier_p=0.01)
+    x[1, 5, 16:32] = 0.0                      # an all-zero block
+    x[2] = 0.0                                # an all-zero tensor
+    packed, scales, g = oracle.quantize(x)
+    xf = x.double().numpy()
+    # zero block and zero tensor
+    assert scales[1, 5, 1] == 0 and np.all(packed[1, 5, 8:16] == 0)
+    assert g[2] == 1.0 and np.all(scales[2] == 0) and np.all(packed[2] == 0)
+    for t in range(2):
+        # the block holding the tensor's largest magnitude gets the top scale 448
+        amax = np.abs(xf[t]).max()
+        assert np.float32(g[t]) == np.float32(np.float32(amax) / np.float32(2688.0))
+        r, c = np.unravel_index(np.abs(xf[t]).argmax(), xf[t].shape)
+        assert scales[t, r, c // 16] == 0x7E
+        # every scale is finite (no NaN code) and no element exceeds 6 * scale * g
+        assert np.all((scales[t] & 0x7F) != 0x7F)
+    w = _decode_with_tables(packed, scales, g)
+    sd = np.repeat(e4m3_torch(scales), 16, axis=-1) * np.asarray(g, np.float64)[:, None, None]
+    assert np.all(np.abs(w) <= 6 * sd)
+    # reconstruction error is at most one E2M1 grid step of the block (spacing <= 2)
+    nz = sd > 0
+    assert np.all(np.abs(xf - w)[nz] <= sd[nz] * 1.0 + 1e-12)
+
+
+def test_dequantize_equals_rounded_exact_product():
+    x = synth.normal_bf16((2, 16, 64), 3, "deq", std=0.5)
+    packed, scales, g = oracle.quantize(x)
+    deq = oracle.dequantize(packed, scales, g)
+    # independent: exact product q*s in fp64 -> times g in fp32 -> bf16 via torch
+    lo, hi = packed & 0xF, packed >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(2, 16, 64)
+    qs = (np.asarray(E2M1_TABLE)[codes] * np.repeat(e4m3_torch(scales), 16, -1)).astype(np.float32)
+    v = qs * np.asarray(g, np.float32)[:, None, None]
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(deq, want)
+
+
+# ------------------------------------------------------------------------------ routing
+def test_route_matches_stable_sort():
+    ids, _ = synth.routing(37, 16, 4, seed=5)
+    ids = ids.numpy().copy()
+    ids[3, 1] = 16     # out of range
+    ids[7, 0] = -1     # out of range
+    ids[9, 2] = ids[9, 3]  # repeated expert within a token
+    counts, offsets, perm, inv, bad = oracle.route(ids, 16)
+    flat = ids.reshape(-1)
+    valid = (flat >= 0) & (flat < 16)
+    assert bad == 2
+    assert np.array_equal(counts, np.bincount(flat[valid], minlength=16))
+    assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    order = np.argsort(np.where(valid, flat, 1 << 20), kind="stable")[: valid.sum()]
+    assert np.array_equal(perm, order)
+    assert np.all(inv[~valid] == -1)
+    assert np.array_equal(perm[inv[valid]], np.nonzero(valid)[0])
+
+
+# ------------------------------------------------------------------------------ MoE
+def _tiny_layer(seed=0, E=8, H=256, I=128):
+    gu, dn = synth.expert_weights_bf16(E, H, I, seed)
+    pg, sg, gg = oracle.quantize(gu)
+    pd, sd, gd = oracle.quantize(dn)
+    return pg, sg, gg, pd, sd, gd
+
+
+def _silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def _bf16_np(v):
+    # fp64 -> fp32 -> bf16 (torch); differs from a single rounding only on exact fp32 ties
+    return torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def test_moe_matches_dense_brute_force_tiny():
+    wl = synth.TINY
+    pg, sg, gg, pd, sd, gd = _tiny_layer(wl.seed, wl.E, wl.H, wl.I)
+    x = synth.activations_bf16(wl.T, wl.H, wl.seed)
+    ids, w = synth.routing(wl.T, wl.E, wl.K, wl.seed)
+    out, out64, bad = oracle.moe_forward(x, ids, w, pg, sg, gg, pd, sd, gd)
+    assert bad == 0
+    # dense: every expert on every token, weighted by a zero-filled gate matrix
+    Wgu = _decode_with_tables(pg, sg, gg)      # [E, 2I, H]
+    Wdn = _decode_with_tables(pd, sd, gd)      # [E, H, I]
+    G = np.zeros((wl.T, wl.E))
+    for t in range(wl.T):
+        for k in range(wl.K):
+            G[t, ids[t, k]] += float(w[t, k])
+    xf = x.double().numpy()
+    a = np.einsum("ejh,th->tej", Wgu, xf)                         # [T, E, 2I]
+    h = _bf16_np(_silu(a[..., : wl.I]) * a[..., wl.I:])             # [T, E, I]
+    y = np.einsum("enj,tej->ten", Wdn, h)                          # [T, E, H]
+    dense = np.einsum("te,ten->tn", G, y)
+    np.testing.assert_allclose(out64, dense, rtol=1e-9, atol=1e-12 * np.abs(dense).max())
+    want_bits = np.array([[oracle.bf16_round(v) for v in row] for row in out64], np.uint16)
+    assert np.array_equal(out, want_bits)
+
+
+def test_moe_single_expert_is_swiglu_mlp():
+    H, I, E = 64, 32, 3
+    pg, sg, gg, pd, sd, gd = _tiny_layer(4, E, H, I)
+    x = synth.activations_bf16(2, H, 4)
+    ids = torch.tensor([[2], [0]], dtype=torch.int32)
+    w = torch.ones((2, 1), dtype=torch.float32)
+    _, out64, _ = oracle.moe_forward(x, ids, w, pg, sg, gg, pd, sd, gd)
+    Wgu = _decode_with_tables(pg, sg, gg)
+    Wdn = _decode_with_tables(pd, sd, gd)
+    for t, e in ((0, 2), (1, 0)):
+        xt = x[t].double().numpy()
+        gate, up = Wgu[e][:I] @ xt, Wgu[e][I:] @ xt
+        want = Wdn[e] @ _bf16_np(_silu(gate) * up)
+        np.testing.assert_allclose(out64[t], want, rtol=1e-10, atol=1e-14)
+
+
+def test_moe_special_cases():
+    H, I, E, K, T = 64, 32, 4, 2, 5
+    pg, sg, gg, pd, sd, gd = _tiny_layer(9, E, H, I)
+    x = synth.activations_bf16(T, H, 9)
+    x[1] = 0.0
+    x[3] = x[2]
+    ids = torch.tensor([[0, 1], [2, 3], [1, 3], [1, 3], [E, 0]], dtype=torch.int32)
+    w = torch.tensor([[0.6, 0.4], [0.5, 0.5], [0.3, 0.7], [0.3, 0.7], [0.9, 0.1]])
+    out, out64, bad = oracle.moe_forward(x, ids, w, pg, sg, gg, pd, sd, gd)
+    assert np.all(out64[1] == 0.0)                      # x = 0 gives 0
+    assert np.array_equal(out[2], out[3])               # identical tokens
+    assert bad == 1                                     # id E is out of range ...
+    ids1 = torch.tensor([[0]], dtype=torch.int32)       # ... and contributes nothing
+    _, ref64, _ = oracle.moe_forward(x[4:5], ids1, torch.tensor([[0.1]]),
+                                     pg, sg, gg, pd, sd, gd)
+    np.testing.assert_allclose(out64[4], ref64[0], rtol=1e-12, atol=0)
+    # swapping the two slots of a token (with their weights) changes nothing but fp64
+    # summation order
+    ids2 = ids[:, [1, 0]].contiguous()
+    w2 = w[:, [1, 0]].contiguous()
+    _, out64b, _ = oracle.moe_forward(x, ids2, w2, pg, sg, gg, pd, sd, gd)
+    np.testing.assert_allclose(out64b, out64, rtol=1e-12, atol=1e-15)
