@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 routed-expert MoE layer on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode1|decode8|decode32|decode64|prefill|codec]
+
+A step is one pass of the whole layer (route -> gate/up + SwiGLU -> down -> combine) over
+one batch.  The default workload is the single-token decode of the H=6144, I=2048, E=256,
+top-8 layer: every step routes a NEW token (synthetic x ~ N(0,1), router logits N(0,1),
+softmax top-8) to 8 of 256 experts whose NVFP4 weights (5.4 GB, N(0,0.02) bf16 quantized by
+the library) stay resident in HBM, so each step reads ~170 MB of expert bytes that are
+not in the 126 MB L2.  Steps are captured in a CUDA graph and timed with CUDA events.
+
+Keys beyond the base contract: `roofline` (dominant kernel, live CUDA-event durations of
+each stage from a second, marked pass), `cpu_baseline` (the CPU oracle on a bounded
+sample, rank 0 at N=1), `e2e` (the same metric through the C ABI with pinned host
+buffers, copies inside the timed region), `clocks`, `gpu_launches`.
+
+--impl reference times the CPU oracle itself on the host cores (the reference arm).
+With torchrun (N>1) every rank runs its own token stream (independent problems, weak
+scaling, no collective on the data path); only a barrier and a max-reduce of the times
+use NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s"
+H, I, E, K = 6144, 2048, 256, 8
+GATEUP_BYTES_PER_EXPERT = 2 * I * (H // 2 + H // 16)      # 14,155,776
+DOWN_BYTES_PER_EXPERT = H * (I // 2 + I // 16)            # 7,077,888
+EXPERT_BYTES = GATEUP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- setup
+def build_layer(nv, device, seed=0):
+    """All 256 experts, bf16 N(0,0.02) drawn on the GPU and quantized by the library."""
+    dev = []
+    for proj, shape in (("w_gu", (2 * I, H)), ("w_dn", (H, I))):
+        x = torch.empty((E,) + shape, dtype=torch.bfloat16, device=device)
+        for e in range(E):
+            x[e] = synth.normal_bf16(shape, seed, proj, e, std=0.02, device=device)
+        dev += list(nv.nvfp4_quantize(x))
+        del x
+    torch.cuda.empty_cache()
+    return dev
+
+
+def workload_of(name):
+    if name.startswith("decode"):
+        T = int(name[len("decode"):])
+        return synth.decode_batch(T) if T > 1 else synth.DECODE_T1
+    if name == "prefill":
+        return synth.PREFILL_T4096
+    if name == "codec":
+        return synth.CODEC_LAYER
+    raise SystemExit(f"unknown workload {name}")
+
+
+def make_batches(wl, n_batches, seed, device):
+    """n_batches independent batches of T tokens: x, ids, w on the device."""
+    T = wl.T
+    xs = synth.activations_bf16(n_batches * T, H, seed, device=device).view(n_batches, T, H)
+    ids, w = synth.routing(n_batches * T, E, K, seed=seed, zipf_bias=wl.zipf_bias)
+    return xs, ids.view(n_batches, T, K).to(device), w.view(n_batches, T, K).to(device)
+
+
+# ----------------------------------------------------------------------------- CPU baseline
+def random_nvfp4_pool(pool, seed=11):
+    """NVFP4 weights for `pool` experts drawn directly as random E2M1 codes and E4M3 scales
+    (for timing the oracle, whose cost does not depend on the values)."""
+    rng = np.random.default_rng(seed)
+    pg = rng.integers(0, 256, (pool, 2 * I, H // 2), dtype=np.uint8)
+    sg = rng.integers(0x30, 0x58, (pool, 2 * I, H // 16), dtype=np.uint8)
+    pd = rng.integers(0, 256, (pool, H, I // 2), dtype=np.uint8)
+    sd = rng.integers(0x30, 0x58, (pool, H, I // 16), dtype=np.uint8)
+    g = np.full((pool,), 1e-3, np.float32)
+    return pg, sg, g, pd, sd, g.copy()
+
+
+def cpu_baseline_decode(n_tokens=4, seed=7):
+    """The CPU oracle on a bounded sample: n_tokens single-token decode steps, each routed
+    to 8 of a pool of 16 experts."""
+    import oracle
+    pool = 16
+    weights = random_nvfp4_pool(pool)
+    ids, w = synth.routing(n_tokens, pool, K, seed=seed)
+    x = synth.activations_bf16(n_tokens, H, seed)
+    t0 = time.perf_counter()
+    for t in range(n_tokens):
+        oracle.moe_forward(x[t:t + 1], ids[t:t + 1], w[t:t + 1], *weights)
+    total = time.perf_counter() - t0
+    return {"value": n_tokens / total, "unit": "tokens/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"{n_tokens} single-token decode steps of the H=6144 I=2048 top-8 layer "
+                      f"(fp64, {oracle.threads()} OpenMP threads)"}
+
+
+# ----------------------------------------------------------------------------- ours
+def run_ours(args, rank, world, device):
+    import bit_quantized_moe_nvfp4_b200 as nv
+    peaks = load_peaks()
+    wl = workload_of(args.workload)
+    if args.workload == "codec":
+        return run_codec(args, nv, rank, world, device, peaks)
+    T = wl.T
+    layer = build_layer(nv, device)
+    # distinct token batches; a graph of G steps is replayed to cover K steps exactly
+    K_steps, W = args.steps, args.warmup
+    G = min(K_steps, args.graph_steps if T <= 64 else 2)
+    n_b = max(G, W)
+    xs, ids, ws_ = make_batches(wl, n_b, seed=1000 + rank, device=device)
+    ws = nv.alloc_moe_workspace(T, H, I, E, K, device)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    path = args.path
+
+    def step(i):
+        nv.moe_nvfp4_forward(xs[i], ids[i], ws_[i], *layer, out=out, workspace=ws, path=path)
+
+    for i in range(W):
+        step(i % n_b)
+    torch.cuda.synchronize()
+
+    # graph of G steps (same kernels, same order as eager calls)
+    stream = torch.cuda.Stream(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        step(0)
+        stream.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(G):
+                step(i)
+    reps, rem = divmod(K_steps, G)
+    tail_graph = None
+    if rem:
+        tail_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tail_graph, stream=stream):
+            for i in range(rem):
+                step(i)
+    graph.replay()
+    torch.cuda.synchronize()
+
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                graph.replay()
+            if tail_graph is not None:
+                tail_graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = ev0.elapsed_time(ev1)
+    ms_total = max_over_ranks(ms_total, world, device)
+    ms_step = ms_total / K_steps
+
+    # marked pass: per-stage durations from events between the kernels
+    n_mark = min(G, 64)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_mark)]
+    mgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(mgraph, stream=stream):
+            for i in range(n_mark):
+                nv.moe_nvfp4_forward_profiled(xs[i], ids[i], ws_[i], *layer, out, ws, marks[i],
+                                              path=path)
+        mgraph.replay()
+    torch.cuda.synchronize()
+    stages = {n: statistics.mean(m[j].elapsed_time(m[j + 1]) for m in marks)
+              for j, n in enumerate(["route", "gate_up", "down", "combine"])}
+    marked_step = statistics.mean(m[0].elapsed_time(m[4]) for m in marks)
+
+    # algorithmic work of the timed steps
+    counts = []
+    for i in range(G):
+        counts.append(len(set(ids[i].flatten().tolist())))
+    uniq = statistics.mean(counts)
+    bytes_step = uniq * EXPERT_BYTES
+    flops_step = 2 * T * K * (3 * H * I)
+    tokens_total = T * K_steps * world
+    value = tokens_total / (ms_total / 1e3)
+
+    if T <= 64:   # HBM-bound: the gate/up GEMV streams 2/3 of the expert bytes
+        gu_ms = stages["gate_up"]
+        achieved = uniq * GATEUP_BYTES_PER_EXPERT / (gu_ms / 1e3) / 1e9
+        roof = {"kernel": "gemv_gateup_kernel (gate/up GEMV + SwiGLU)", "bound": "hbm",
+                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_bytes": uniq * GATEUP_BYTES_PER_EXPERT,
+                "peak_source": peaks["source"] + " (burst copy)"}
+    else:
+        gu_ms = stages["gate_up"]
+        fl = 2 * T * K * (2 * I * H)
+        achieved = fl / (gu_ms / 1e3) / 1e12
+        pk = peaks["bf16_tflops"]
+        roof = {"kernel": "gemm_gateup (tcgen05 grouped GEMM + SwiGLU)", "bound": "tensor",
+                "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
+                "traffic": None, "algorithmic_flops": fl,
+                "peak_source": peaks["source"] + " (cuBLAS bf16 burst)"}
+
+    # end to end through the C ABI with pinned host buffers
+    e2e = run_e2e(nv, layer, wl, args, device, ws, path)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": K_steps, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) bf16 weights quantized to NVFP4)",
+        "config": {"workload": wl.name, "T": T, "H": H, "I": I, "E": E, "K": K,
+                   "weights": "NVFP4 (E2M1 + E4M3 per 16 + fp32 per tensor), 5.4 GB resident",
+                   "l2": "inputs larger than L2: every step routes new tokens over 5.4 GB of "
+                         "expert weights (>126 MB L2)",
+                   "timing": f"CUDA graph of {G} steps replayed, CUDA events",
+                   "path": {0: "auto", 1: "gemv", 2: "gemm"}[path],
+                   "parallelism": f"{world} independent replica(s), no data-path collective"},
+        "hbm_gbs_step": bytes_step / (ms_step / 1e3) / 1e9,
+        "tflops_step": flops_step / (ms_step / 1e3) / 1e12,
+        "unique_experts_per_step": uniq,
+        "stages_ms": stages, "marked_step_ms": marked_step,
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": 4 * K_steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_decode(args.cpu_tokens)
+    return line
+
+
+def run_e2e(nv, layer, wl, args, device, ws, path):
+    """Same metric through the public API with host buffers: per step, copy the step's
+    x / ids / weights from pinned host memory, run the layer, copy the output back."""
+    T = wl.T
+    n = min(args.e2e_steps, 256)
+    xs = synth.activations_bf16(n * T, H, 77).view(n, T, H).pin_memory()
+    ids, w = synth.routing(n * T, E, K, seed=77, zipf_bias=wl.zipf_bias)
+    ids = ids.view(n, T, K).pin_memory()
+    w = w.view(n, T, K).pin_memory()
+    out_h = torch.empty((n, T, H), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    idd = torch.empty((T, K), dtype=torch.int32, device=device)
+    wd = torch.empty((T, K), dtype=torch.float32, device=device)
+    od = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+
+    def one(i):
+        xd.copy_(xs[i], non_blocking=True)
+        idd.copy_(ids[i], non_blocking=True)
+        wd.copy_(w[i], non_blocking=True)
+        nv.moe_nvfp4_forward(xd, idd, wd, *layer, out=od, workspace=ws, path=path)
+        out_h[i].copy_(od, non_blocking=True)
+
+    for i in range(min(3, n)):
+        one(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        one(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    return {"value": n * T / (ms / 1e3), "unit": "tokens/s", "steps": n,
+            "h2d_bytes_per_step": T * H * 2 + T * K * 4 * 2, "d2h_bytes_per_step": T * H * 2}
+
+
+def run_codec(args, nv, rank, world, device, peaks):
+    """Whole-layer quantize + dequantize of all 256 experts (gate/up and down)."""
+    wl = synth.CODEC_LAYER
+    xs = {}
+    for proj, shape in (("w_gu", (2 * I, H)), ("w_dn", (H, I))):
+        x = torch.empty((E,) + shape, dtype=torch.bfloat16, device=device)
+        for e in range(E):
+            x[e] = synth.normal_bf16(shape, wl.seed, proj, e, std=0.02, device=device,
+                                     outlier_p=wl.outlier_p)
+        xs[proj] = x
+    outs = {p: nv.nvfp4_quantize(x) for p, x in xs.items()}
+    deq = {p: torch.empty_like(x) for p, x in xs.items()}
+    elts = sum(x.numel() for x in xs.values())
+
+    def q():
+        for p, x in xs.items():
+            nv.nvfp4_quantize(x, *outs[p])
+
+    def d():
+        for p in xs:
+            nv.nvfp4_dequantize(*outs[p], out=deq[p])
+
+    res = {}
+    for name, fn in (("quantize", q), ("dequantize", d)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        gbs = elts * 2.5625 / (ms / 1e3) / 1e9
+        res[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]}
+    return {"metric": "NVFP4 codec GB/s (whole layer)", "value": res["quantize"]["GB/s"],
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": res["quantize"]["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "elements": elts},
+            "codec": res, "gpu_launches": 2 * 2 * args.steps}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The CPU oracle as it stands, on the host cores: each step is one single-token decode
+    step of the same layer (8 experts).  NVFP4 weights for a pool of experts are drawn
+    directly as random codes and scales (the oracle's cost does not depend on values)."""
+    import oracle
+    pool = 16
+    pg, sg, gg, pd, sd, gd = random_nvfp4_pool(pool)
+    n = args.steps + args.warmup
+    x = synth.activations_bf16(n, H, 5)
+    ids, w = synth.routing(n, pool, K, seed=5)
+    times = []
+    for i in range(n):
+        t0 = time.perf_counter()
+        oracle.moe_forward(x[i:i + 1], ids[i:i + 1], w[i:i + 1], pg, sg, gg, pd, sd, gd)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times)
+    v = len(times) / sec
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": synth.DECODE_T1.name},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(),
+                             "kind": "oracle",
+                             "sample": "each step one single-token decode step (8 experts)"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- plumbing
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8192)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode1")
+    ap.add_argument("--path", type=int, default=0)
+    ap.add_argument("--graph-steps", type=int, default=512)
+    ap.add_argument("--e2e-steps", type=int, default=256)
+    ap.add_argument("--cpu-tokens", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=device,
+                                             timeout=datetime.timedelta(seconds=300))
+    try:
+        line = run_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

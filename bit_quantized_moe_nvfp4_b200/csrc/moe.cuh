@@ -1,0 +1,76 @@
+// moe.cuh -- arguments and workspace layout shared by the MoE forward kernels.
+#pragma once
+#include "route.cuh"
+
+namespace nvfp4 {
+
+// Everything one forward call needs on the device.  Weight pointers are the caller's;
+// the int32 / bf16 / fp32 scratch arrays live in the caller's workspace.
+struct MoeArgs {
+  // inputs
+  const __nv_bfloat16 *x;     // [T, H]
+  const int32_t *ids;         // [T, K]
+  const float *w;             // [T, K]
+  const uint8_t *w_gu;        // [E, 2I, H/2]
+  const uint8_t *s_gu;        // [E, 2I, H/16]
+  const float *g_gu;          // [E]
+  const uint8_t *w_dn;        // [E, H, I/2]
+  const uint8_t *s_dn;        // [E, H, I/16]
+  const float *g_dn;          // [E]
+  __nv_bfloat16 *out;         // [T, H]
+  int64_t T, H, I, E, K;
+  // workspace
+  int32_t *flag;              // [1] error bits
+  int32_t *n_active;          // [1]
+  int32_t *counts;            // [E]
+  int32_t *offsets;           // [E+1]
+  int32_t *active;            // [E]
+  int32_t *tile_prefix;       // [E+1]
+  int32_t *perm;              // [T*K]  pair index t*K+k, grouped by expert
+  int32_t *inv;               // [T*K]  position of pair t*K+k in perm
+  __nv_bfloat16 *h;           // [T*K, I]   SwiGLU output, rows in perm order
+  float *y;                   // [T*K, H]   w * g_dn * (W_dn h), rows in perm order
+  __nv_bfloat16 *xs;          // [T*K + pad, H]  x gathered in perm order (GEMM path)
+};
+
+// Workspace carve-up (byte offsets, each 256-aligned).
+struct WorkspaceLayout {
+  size_t flag, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, total;
+};
+WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
+constexpr int kGatherPadRows = 256;
+
+// GEMV path (decode.cu) and combine (combine.cu)
+int launch_gemv_gateup(const MoeArgs &a, cudaStream_t s);
+int launch_gemv_down(const MoeArgs &a, cudaStream_t s);
+int launch_combine(const MoeArgs &a, cudaStream_t s);
+// GEMM path (gemm.cu)
+int launch_gemm_gateup(const MoeArgs &a, cudaStream_t s);   // gather + gate/up + SwiGLU
+int launch_gemm_down(const MoeArgs &a, cudaStream_t s);
+int gemm_tile_n();
+
+// Launch with programmatic dependent launch enabled (the kernel must call pdl_wait()
+// before it reads what the previous kernel wrote).
+template <typename Kern, typename... Args>
+int launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return NVFP4_ECUDA;
+  }
+  return NVFP4_OK;
+}
+
+__device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+
+}  // namespace nvfp4

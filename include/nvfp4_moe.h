@@ -1,0 +1,180 @@
+/*
+ * nvfp4_moe.h -- C ABI of the NVFP4 routed-expert MoE library (sm_100a).
+ *
+ * What the library computes is defined on page "GLM-5-NVFP4-MTP":
+ *   "Model Description" -- the expert weights are NVFP4: 4-bit values with one FP8 scale per
+ *                          16 consecutive elements; each MoE layer has 256 experts, 8 active
+ *                          per token.
+ *   "What's quantized"  -- only the routed experts' gate, up and down projections are NVFP4.
+ * The format is fixed as: E2M1 elements, E4M3 ("FN", finite) block scales, one fp32 global
+ * scale g per tensor, block scale = (block amax / 6) / g rounded to E4M3 (nearest, ties to
+ * even, saturating at 448), g = tensor amax / (6 * 448) (1 for an all-zero tensor).
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers owned by the caller unless a parameter says "host".
+ *     The library never allocates, frees or keeps memory; scratch comes from a caller
+ *     workspace sized by the matching *_workspace_size() query.
+ *   - Calls are asynchronous on `stream`: they enqueue kernels and return without waiting.
+ *   - The return value is a status: NVFP4_OK (0) on success.  On a negative status nothing
+ *     was enqueued (argument checks run before any launch), except NVFP4_ECUDA, which reports
+ *     a failed launch; nvfp4_last_cuda_error() then names the CUDA error.
+ *   - Layouts are row-major.  A packed row stores element 2j in the LOW nibble of byte j and
+ *     element 2j+1 in the HIGH nibble.  Block scales run along the contiguous dimension.
+ *   - The library keeps no global state apart from a per-thread copy of the last CUDA error;
+ *     calls on different streams may run concurrently if their workspaces differ.
+ */
+#ifndef NVFP4_MOE_H
+#define NVFP4_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status codes */
+#define NVFP4_OK 0
+#define NVFP4_EINVAL -1      /* null pointer, negative or zero dimension, bad path value */
+#define NVFP4_ESHAPE -2      /* a dimension that must be a multiple of 16/32 is not, or a
+                                size above a documented limit */
+#define NVFP4_EWORKSPACE -3  /* workspace pointer null or smaller than the query says */
+#define NVFP4_ECUDA -4       /* a kernel launch failed; see nvfp4_last_cuda_error() */
+
+/* Human-readable name of a status code (static string). */
+NVFP4_API const char *nvfp4_status_string(int status);
+
+/* Text of the last CUDA error seen by a call on this host thread ("no error" if none). */
+NVFP4_API const char *nvfp4_last_cuda_error(void);
+
+/* ---------------------------------------------------------------- codec */
+
+/* Bytes of workspace nvfp4_quantize needs (a per-tensor amax accumulator). */
+NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t n_tensors, int64_t rows, int64_t cols);
+
+/* Quantize n_tensors bf16 tensors of shape [rows, cols] to NVFP4 (page "GLM-5-NVFP4-MTP",
+ * "Model Description": 4-bit values, one FP8 scale per 16 elements).
+ *   x            [n_tensors, rows, cols] bf16
+ *   packed       [n_tensors, rows, cols/2] E2M1 codes, two per byte (low nibble first)
+ *   scales       [n_tensors, rows, cols/16] E4M3 codes
+ *   global_scale [n_tensors] fp32, g = amax / 2688 (1.0 for an all-zero tensor)
+ * Per 16-element block: s = (amax_b / 6) / g -> E4M3 (nearest, ties to even, saturating);
+ * d = decoded s * g; code_i = E2M1(x_i / d) (nearest, ties to even, saturating at 6, sign
+ * kept, so a small negative value gives 0x8); all codes 0 when d == 0.  Every step is an
+ * IEEE fp32 operation rounded to nearest even, so results are reproducible bit for bit.
+ * Requires cols % 32 == 0.  NaN/Inf inputs give unspecified codes.
+ * Alignment: x 16 bytes, packed and global_scale 4 bytes, workspace 4 bytes.
+ * Errors: EINVAL (null pointer, dimension <= 0, misaligned pointer), ESHAPE (cols % 32 != 0),
+ * EWORKSPACE (ws_bytes < nvfp4_quantize_workspace_size). */
+NVFP4_API int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t rows, int64_t cols,
+                   uint8_t *packed, uint8_t *scales, float *global_scale,
+                   void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Dequantize NVFP4 to bf16: out = bf16( fp32(e2m1 * e4m3) * g ), the first product exact,
+ * the multiply by g rounded once in fp32, then rounded to bf16 (nearest even).
+ * Shapes as in nvfp4_quantize; requires cols % 32 == 0.  Alignment: packed and out 16
+ * bytes, scales 2 bytes.  Errors: EINVAL (null or misaligned pointer), ESHAPE. */
+NVFP4_API int nvfp4_dequantize(const uint8_t *packed, const uint8_t *scales, const float *global_scale,
+                     int64_t n_tensors, int64_t rows, int64_t cols, __nv_bfloat16 *out,
+                     cudaStream_t stream);
+
+/* Scalar format casts, element by element, exactly as the quantizer takes them:
+ * e4m3[i] = E4M3(in[i]) and e2m1[i] = E2M1(in[i]) (nearest, ties to even, saturating,
+ * sign kept; one code per byte in the low nibble for E2M1).  Either output may be NULL.
+ * Errors: EINVAL (in NULL or n <= 0). */
+NVFP4_API int nvfp4_cast_f32(const float *in, int64_t n, uint8_t *e4m3, uint8_t *e2m1,
+                   cudaStream_t stream);
+
+/* ---------------------------------------------------------------- MoE layer */
+
+/* Routed-expert MoE MLP of one layer, run directly from NVFP4 expert weights (page
+ * "GLM-5-NVFP4-MTP", "Model Description": 256 experts, 8 active per token; "What's
+ * quantized": gate, up and down projections are NVFP4).  For token t:
+ *   out[t] = sum over k = 0..K-1 of topk_w[t,k] * y_k, with e = topk_ids[t,k] and
+ *   a   = g_gu[e] * (W_gu[e] x_t)        2I values: rows 0..I-1 gate, rows I..2I-1 up
+ *   h_j = bf16( silu(a_j) * a_{I+j} )     SwiGLU, rounded to bf16
+ *   y_k = g_dn[e] * (W_dn[e] h)           H values
+ * where each weight is its exact NVFP4 value e2m1 * e4m3 (products accumulate in fp32).
+ * Ids outside [0, E) contribute nothing and set the workspace error flag
+ * (moe_nvfp4_read_error_flag).  A repeated id within a token counts once per slot.
+ *   x        [T, H] bf16            topk_ids [T, K] int32      topk_w [T, K] fp32
+ *   w_gu     [E, 2I, H/2] u8        s_gu [E, 2I, H/16] E4M3    g_gu [E] fp32
+ *   w_dn     [E, H, I/2] u8         s_dn [E, H, I/16] E4M3     g_dn [E] fp32
+ *   out      [T, H] bf16
+ * Limits: H % 64 == 0, I % 64 == 0, 1 <= K <= 16, E <= 1024, T*K < 2^31.
+ * Alignment: x, w_gu, w_dn, out and workspace 16 bytes; s_gu, s_dn 2 bytes (EINVAL /
+ * EWORKSPACE otherwise).
+ * The call picks a memory-bound GEMV path for small T and a tensor-core grouped GEMM path
+ * otherwise; both compute the same function.  It never synchronises with the host and
+ * may be captured in a CUDA graph.
+ * Errors: EINVAL, ESHAPE, EWORKSPACE (ws_bytes < moe_nvfp4_workspace_size), ECUDA. */
+NVFP4_API size_t moe_nvfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
+
+NVFP4_API int moe_nvfp4_forward(const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w,
+                      int64_t T, int64_t H, int64_t I, int64_t E, int64_t K,
+                      const uint8_t *w_gu, const uint8_t *s_gu, const float *g_gu,
+                      const uint8_t *w_dn, const uint8_t *s_dn, const float *g_dn,
+                      __nv_bfloat16 *out, void *workspace, size_t ws_bytes,
+                      cudaStream_t stream);
+
+/* Paths of moe_nvfp4_forward_path. */
+#define NVFP4_PATH_AUTO 0     /* what moe_nvfp4_forward does */
+#define NVFP4_PATH_GEMV 1     /* dequant-fused grouped GEMV (CUDA cores), any T */
+#define NVFP4_PATH_GEMM 2     /* dequant-to-shared-memory grouped GEMM (tcgen05), any T */
+
+/* moe_nvfp4_forward with the path chosen by the caller (same arguments, same result up
+ * to fp32 summation order).  Errors as moe_nvfp4_forward, plus EINVAL for a bad path. */
+NVFP4_API int moe_nvfp4_forward_path(const __nv_bfloat16 *x, const int32_t *topk_ids,
+                           const float *topk_w, int64_t T, int64_t H, int64_t I, int64_t E,
+                           int64_t K, const uint8_t *w_gu, const uint8_t *s_gu,
+                           const float *g_gu, const uint8_t *w_dn, const uint8_t *s_dn,
+                           const float *g_dn, __nv_bfloat16 *out, void *workspace,
+                           size_t ws_bytes, int path, cudaStream_t stream);
+
+/* moe_nvfp4_forward_path with timing marks, for measurement.  stage_events points to five
+ * cudaEvent_t (created by the caller, timing enabled) that are recorded on `stream`:
+ * [0] before the route step, [1] after it, [2] after the gate/up + SwiGLU step, [3] after
+ * the down step, [4] after the combine.  The events sit between the kernels, so the
+ * kernels do not overlap their neighbours as they do in an unmarked call.
+ * Errors as moe_nvfp4_forward_path, plus EINVAL for a null event. */
+NVFP4_API int moe_nvfp4_forward_profiled(const __nv_bfloat16 *x, const int32_t *topk_ids,
+                                         const float *topk_w, int64_t T, int64_t H, int64_t I,
+                                         int64_t E, int64_t K, const uint8_t *w_gu,
+                                         const uint8_t *s_gu, const float *g_gu,
+                                         const uint8_t *w_dn, const uint8_t *s_dn,
+                                         const float *g_dn, __nv_bfloat16 *out,
+                                         void *workspace, size_t ws_bytes, int path,
+                                         void *const *stage_events, cudaStream_t stream);
+
+/* Copy the workspace error flag to *host_flag (host pointer) and wait for it:
+ * 0 = no error, bit 0 = an id outside [0, E) was met, bit 1 = a device-side wait gave up.
+ * The flag is cleared by the next moe_nvfp4_forward on that workspace.  Synchronises
+ * `stream`.  Errors: EINVAL, ECUDA. */
+NVFP4_API int moe_nvfp4_read_error_flag(const void *workspace, int32_t *host_flag, cudaStream_t stream);
+
+/* The token permutation step on its own (the first step of moe_nvfp4_forward):
+ *   counts[e]  = number of (t, k) with topk_ids[t,k] == e                  [E]
+ *   offsets    = exclusive prefix sum of counts                             [E+1]
+ *   perm       = flat pair indices t*K+k grouped by expert, ascending within
+ *                an expert; entries past offsets[E] are left unwritten      [T*K]
+ *   inv[t*K+k] = position of that pair in perm, -1 for an out-of-range id  [T*K]
+ *   error_flag = bit 0 set when an id is out of range (may be NULL)         [1]
+ * Limits: E <= 1024, 1 <= K <= 16, T*K < 2^31.  Errors: EINVAL, ESHAPE, ECUDA. */
+NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int64_t E,
+                    int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
+                    int32_t *error_flag, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_MOE_H */

@@ -1,0 +1,129 @@
+"""The C ABI loads on a machine without a GPU, exports every entry point the header
+declares, and rejects bad arguments with status codes before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4_moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_quantized_moe_nvfp4_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^NVFP4_API[^;(]*?\b(\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for want in ("nvfp4_quantize", "nvfp4_dequantize", "moe_nvfp4_forward",
+                 "moe_nvfp4_workspace_size", "moe_nvfp4_route", "nvfp4_status_string"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    lib.nvfp4_status_string.restype = ctypes.c_char_p
+    for code, word in ((0, b"OK"), (-1, b"EINVAL"), (-2, b"ESHAPE"), (-3, b"EWORKSPACE"),
+                       (-4, b"ECUDA")):
+        assert word in lib.nvfp4_status_string(code)
+
+
+def test_workspace_queries(lib):
+    lib.moe_nvfp4_workspace_size.restype = ctypes.c_size_t
+    lib.moe_nvfp4_workspace_size.argtypes = [ctypes.c_int64] * 5
+    small = lib.moe_nvfp4_workspace_size(1, 6144, 2048, 256, 8)
+    big = lib.moe_nvfp4_workspace_size(4096, 6144, 2048, 256, 8)
+    assert 0 < small < big
+    # the prefill scratch: gathered x, h and the fp32 per-pair outputs dominate
+    TK = 4096 * 8
+    assert big >= TK * (2 * 6144 + 2 * 2048 + 4 * 6144)
+    assert lib.moe_nvfp4_workspace_size(0, 6144, 2048, 256, 8) == 0
+
+
+def _fwd_argtypes(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    f = lib.moe_nvfp4_forward_path
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, I64, I64, I64, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_size_t,
+                  ctypes.c_int, P]
+    return f
+
+
+def test_forward_argument_checks_run_before_cuda(lib):
+    f = _fwd_argtypes(lib)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails its checks
+    good = dict(T=1, H=6144, I=2048, E=256, K=8)
+
+    def call(ptr=fake, ws=fake, ws_bytes=1 << 40, path=0, **over):
+        d = dict(good, **over)
+        return f(ptr, ptr, ptr, d["T"], d["H"], d["I"], d["E"], d["K"], ptr, ptr, ptr, ptr,
+                 ptr, ptr, ptr, ws, ws_bytes, path, None)
+
+    assert call(ptr=None) == -1            # null pointers
+    assert call(T=0) == -1
+    assert call(path=7) == -1
+    assert call(H=6100) == -2              # not a multiple of 64
+    assert call(I=2040) == -2
+    assert call(K=17) == -2
+    assert call(E=2048) == -2
+    assert call(ws=None) == -3
+    assert call(ws_bytes=16) == -3
+
+
+def test_codec_argument_checks_run_before_cuda(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    q = lib.nvfp4_quantize
+    q.restype = ctypes.c_int
+    q.argtypes = [P, I64, I64, I64, P, P, P, P, ctypes.c_size_t, P]
+    fake = ctypes.c_void_p(1 << 20)
+    assert q(None, 1, 16, 32, fake, fake, fake, fake, 1 << 20, None) == -1
+    assert q(fake, 1, 16, 48, fake, fake, fake, fake, 1 << 20, None) == -2
+    assert q(fake, 1, 16, 32, fake, fake, fake, None, 0, None) == -3
+    d = lib.nvfp4_dequantize
+    d.restype = ctypes.c_int
+    d.argtypes = [P, P, P, I64, I64, I64, P, P]
+    assert d(fake, fake, fake, 1, 16, 40, fake, None) == -2
+    assert d(fake, None, fake, 1, 16, 32, fake, None) == -1
+
+
+def test_route_argument_checks_run_before_cuda(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    r = lib.moe_nvfp4_route
+    r.restype = ctypes.c_int
+    r.argtypes = [P, I64, I64, I64, P, P, P, P, P, P]
+    fake = ctypes.c_void_p(1 << 20)
+    assert r(None, 4, 2, 8, fake, fake, fake, fake, None, None) == -1
+    assert r(fake, 4, 17, 8, fake, fake, fake, fake, None, None) == -2
+    assert r(fake, 4, 2, 4096, fake, fake, fake, fake, None, None) == -2
+
+
+def test_oracle_and_product_share_no_code():
+    """The product never imports, links or includes the oracle, and the oracle never
+    imports or includes the product."""
+    pkg = os.path.join(ROOT, "bit_quantized_moe_nvfp4_b200")
+    bad_in_product = re.compile(r"^\s*(import|from)\s+oracle\b|liboracle|nvfp4_oracle", re.M)
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".cu", ".cuh", ".py", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not bad_in_product.search(text), fn
+    bad_in_oracle = re.compile(
+        r"^\s*(import|from)\s+bit_quantized_moe_nvfp4_b200\b|#include\s+\"[^\"]*(csrc|nvfp4_moe)",
+        re.M)
+    for fn in os.listdir(os.path.join(ROOT, "oracle")):
+        if fn.endswith((".c", ".h", ".py")):
+            text = open(os.path.join(ROOT, "oracle", fn)).read()
+            assert not bad_in_oracle.search(text), fn

@@ -1,0 +1,157 @@
+"""MoE forward on the GPU against the CPU oracle (both kernel paths).
+
+Bar: relative Frobenius error <= 2e-3 and max abs error <= 1e-2 * max|ref| against the
+oracle's bf16 output (bf16 output, fp32 accumulation).  At full layer size the oracle
+computes sampled tokens one by one; the weights it reads are quantized by the oracle from
+the same seeded bf16 draws, after checking they equal the GPU quantizer's bytes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import Layer, compare_moe
+
+pytestmark = pytest.mark.gpu
+
+PATHS = [1, 2]   # GEMV (CUDA cores), GEMM (tcgen05)
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import bit_quantized_moe_nvfp4_b200 as m
+    return m
+
+
+def run(nv, layer, x, ids, w, path):
+    return nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *layer.dev, path=path)
+
+
+@pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
+def test_tiny_layer(nv, path):
+    wl = synth.TINY
+    layer = Layer(wl.E, wl.H, wl.I, wl.seed)
+    x = synth.activations_bf16(wl.T, wl.H, wl.seed)
+    ids, w = synth.routing(wl.T, wl.E, wl.K, wl.seed)
+    out = run(nv, layer, x, ids, w, path)
+    ref, ref64, _ = layer.oracle_forward(x, ids, w)
+    compare_moe(out, ref, ref64)
+
+
+@pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
+@pytest.mark.parametrize("T", [1, 5, 37, 200])
+def test_small_layer_many_shapes(nv, path, T):
+    E, H, I, K = 16, 192, 128, 4
+    layer = Layer(E, H, I, seed=T, outlier_p=0.01)
+    x = synth.activations_bf16(T, H, T)
+    ids, w = synth.routing(T, E, K, seed=T, zipf_bias=1.5)
+    out = run(nv, layer, x, ids, w, path)
+    ref, ref64, _ = layer.oracle_forward(x, ids, w)
+    compare_moe(out, ref, ref64)
+
+
+@pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
+def test_edge_cases(nv, path):
+    """One expert takes every token, most experts are empty, a zero token, a repeated id
+    within a token, and an out-of-range id (contributes nothing, raises the flag)."""
+    E, H, I, K, T = 6, 128, 64, 3, 41
+    layer = Layer(E, H, I, seed=2)
+    x = synth.activations_bf16(T, H, 2)
+    x[7] = 0.0
+    ids = torch.zeros((T, K), dtype=torch.int32)
+    ids[:, 1] = 3
+    ids[:, 2] = 3               # repeated id
+    ids[5, 2] = E               # out of range
+    w = torch.full((T, K), 1.0 / K)
+    ws = nv.alloc_moe_workspace(T, H, I, E, K)
+    out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *layer.dev, workspace=ws,
+                               path=path)
+    assert nv.moe_nvfp4_read_error_flag(ws) & 1
+    ref, ref64, bad = layer.oracle_forward(x, ids, w)
+    assert bad == 1
+    compare_moe(out, ref, ref64)
+    assert torch.all(out[7] == 0)
+    # a clean call on the same workspace clears the flag
+    ids[5, 2] = 1
+    nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *layer.dev, workspace=ws, path=path)
+    assert nv.moe_nvfp4_read_error_flag(ws) == 0
+
+
+# ----------------------------------------------------------------------------- full size
+class FullLayer:
+    """All 256 experts of the H=6144, I=2048 layer on the GPU, quantized by the GPU
+    quantizer (N(0, 0.02) bf16 weights)."""
+
+    def __init__(self, nv, seed=0):
+        wl = synth.DECODE_T1
+        self.E, self.H, self.I, self.seed = wl.E, wl.H, wl.I, seed
+        self._cache = {}
+        self.dev = []
+        for proj, shape in (("w_gu", (2 * self.I, self.H)), ("w_dn", (self.H, self.I))):
+            x = torch.empty((self.E,) + shape, dtype=torch.bfloat16, device="cuda")
+            for e in range(self.E):
+                x[e] = synth.normal_bf16(shape, seed, proj, e, std=0.02, device="cuda")
+            self.dev += list(nv.nvfp4_quantize(x))
+            del x
+        torch.cuda.empty_cache()
+
+    def oracle_inputs(self, experts):
+        """Oracle-quantized weights of the listed experts (after checking the GPU bytes)."""
+        key = tuple(experts)
+        if key in self._cache:
+            return self._cache[key]
+        host = []
+        for pi, (proj, shape) in enumerate((("w_gu", (2 * self.I, self.H)),
+                                            ("w_dn", (self.H, self.I)))):
+            x = torch.stack([synth.normal_bf16(shape, self.seed, proj, e, std=0.02,
+                                               device="cuda").cpu() for e in experts])
+            rp, rs, rg = oracle.quantize(x)
+            ix = torch.tensor(experts, device="cuda")
+            assert np.array_equal(self.dev[3 * pi][ix].cpu().numpy(), rp)
+            assert np.array_equal(self.dev[3 * pi + 1][ix].cpu().numpy(), rs)
+            assert np.array_equal(self.dev[3 * pi + 2][ix].cpu().numpy().view(np.uint32),
+                                  rg.view(np.uint32))
+            host += [rp, rs, rg]
+        self._cache = {key: host}
+        return host
+
+
+@pytest.fixture(scope="module")
+def full(nv):
+    return FullLayer(nv)
+
+
+def _check_sampled(full, x, ids, w, out, tokens):
+    for t in tokens:
+        experts = sorted(set(int(e) for e in ids[t]))
+        remap = {e: i for i, e in enumerate(experts)}
+        ids_t = torch.tensor([[remap[int(e)] for e in ids[t]]], dtype=torch.int32)
+        host = full.oracle_inputs(experts)
+        ref, ref64, bad = oracle.moe_forward(x[t:t + 1], ids_t, w[t:t + 1], *host)
+        assert bad == 0
+        compare_moe(out[t:t + 1], ref, ref64)
+
+
+@pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_full_layer_decode(nv, full, path, T):
+    wl = synth.decode_batch(T)
+    x = synth.activations_bf16(T, wl.H, 100 + T)
+    ids, w = synth.routing(T, wl.E, wl.K, seed=100 + T)
+    out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *full.dev, path=path)
+    torch.cuda.synchronize()
+    _check_sampled(full, x, ids, w, out, tokens=[0, T - 1] if T > 1 else [0])
+
+
+@pytest.mark.parametrize("path", [2, 0], ids=["gemm", "auto"])
+def test_full_layer_prefill(nv, full, path):
+    wl = synth.PREFILL_T4096
+    x = synth.activations_bf16(wl.T, wl.H, wl.seed)
+    ids, w = synth.routing(wl.T, wl.E, wl.K, seed=wl.seed, zipf_bias=wl.zipf_bias)
+    out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *full.dev, path=path)
+    torch.cuda.synchronize()
+    _check_sampled(full, x, ids, w, out, tokens=[0, 2049])
+    # the rest of the batch: cheap invariants over every token
+    o = out.float()
+    assert torch.isfinite(o).all()
+    assert (o.abs().amax(dim=1) > 0).all()
