@@ -40,7 +40,8 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "MoE-layer tokens/s"
-H, I, E, K = 6144, 2048, 256, 8
+H, I, K = 6144, 2048, 8
+E = 256
 GATEUP_BYTES_PER_EXPERT = 2 * I * (H // 2 + H // 16)      # 14,155,776
 DOWN_BYTES_PER_EXPERT = H * (I // 2 + I // 16)            # 7,077,888
 EXPERT_BYTES = GATEUP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT
@@ -236,6 +237,10 @@ def run_ours(args, rank, world, device):
     # marked pass: per-stage durations from events between the kernels
     n_mark = min(G, 64)
     marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_mark)]
+    for m in marks:          # torch creates the CUDA event on its first record
+        for e in m:
+            e.record()
+    torch.cuda.synchronize()
     mgraph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(mgraph, stream=stream):
@@ -284,7 +289,8 @@ def run_ours(args, rank, world, device):
         "steps": K_steps, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) bf16 weights quantized to NVFP4)",
-        "config": {"workload": wl.name, "T": T, "H": H, "I": I, "E": E, "K": K,
+        "config": {"workload": wl.name if E == 256 else wl.name.replace("E=256", f"E={E}"),
+                   "T": T, "H": H, "I": I, "E": E, "K": K,
                    "weights": "NVFP4 (E2M1 + E4M3 per 16 + fp32 per tensor), 5.4 GB resident",
                    "l2": "inputs larger than L2: every step routes new tokens over 5.4 GB of "
                          "expert weights (>126 MB L2)",
@@ -297,7 +303,7 @@ def run_ours(args, rank, world, device):
         "stages_ms": stages, "marked_step_ms": marked_step,
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": 4 * K_steps,
+        "gpu_launches": (2 if (path == 1 or (path == 0 and T <= 64)) else 4) * K_steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -443,9 +449,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--cpu-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=256,
+                    help="experts in the layer (a smaller layer is only for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    global E
+    E = args.experts
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -59,7 +59,7 @@ WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // Token count at or below which the GEMV kernels run (few tokens per expert).
-constexpr int64_t kGemvMaxTokens = int64_t(1) << 40;
+constexpr int64_t kGemvMaxTokens = 64;
 
 }  // namespace nvfp4
 
@@ -84,9 +84,16 @@ extern "C" size_t moe_nvfp4_workspace_size(int64_t T, int64_t H, int64_t I, int6
   return workspace_layout(T, H, I, E, K).total;
 }
 
+// Record a timing mark.  Under stream capture an event record becomes a graph node only
+// when recorded as an external event.
 static int record(cudaEvent_t const *ev, int i, cudaStream_t s) {
   if (!ev) return NVFP4_OK;
-  cudaError_t e = cudaEventRecord(ev[i], s);
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &st);
+  if (e == cudaSuccess)
+    e = (st == cudaStreamCaptureStatusActive)
+            ? cudaEventRecordWithFlags(ev[i], s, cudaEventRecordExternal)
+            : cudaEventRecord(ev[i], s);
   if (e != cudaSuccess) {
     set_last_cuda_error(e);
     return NVFP4_ECUDA;
@@ -108,7 +115,7 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   if (H % 64 || I % 64 || K > 16 || E > kMaxExperts || T * K >= (int64_t(1) << 31))
     return NVFP4_ESHAPE;
   if (!aligned16(x) || !aligned16(w_gu) || !aligned16(w_dn) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(s_gu) & 1) || (reinterpret_cast<uintptr_t>(s_dn) & 1))
+      !aligned16(s_gu) || !aligned16(s_dn))
     return NVFP4_EINVAL;
   const WorkspaceLayout L = workspace_layout(T, H, I, E, K);
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return NVFP4_EWORKSPACE;
@@ -142,7 +149,21 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   a.y = reinterpret_cast<float *>(ws + L.y);
   a.xs = reinterpret_cast<__nv_bfloat16 *>(ws + L.xs);
 
-  if (path == NVFP4_PATH_AUTO) path = (T <= kGemvMaxTokens) ? NVFP4_PATH_GEMV : NVFP4_PATH_GEMM;
+  if (path == NVFP4_PATH_AUTO)
+    path = (T <= kGemvMaxTokens && gemv_supported(T, H, I, K)) ? NVFP4_PATH_GEMV
+                                                               : NVFP4_PATH_GEMM;
+  if (path == NVFP4_PATH_GEMV && !gemv_supported(T, H, I, K)) return NVFP4_ESHAPE;
+
+  if (path == NVFP4_PATH_GEMV) {
+    // two kernels: routing is recomputed inside each, the combine is fused into the second
+    if (int s = record(ev, 0, stream)) return s;
+    if (int s = record(ev, 1, stream)) return s;
+    if (int s = launch_gemv_gateup(a, stream)) return s;
+    if (int s = record(ev, 2, stream)) return s;
+    if (int s = launch_gemv_down(a, stream)) return s;
+    if (int s = record(ev, 3, stream)) return s;
+    return record(ev, 4, stream);
+  }
 
   RouteArgs r = {};
   r.ids = topk_ids;
@@ -155,20 +176,14 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   r.flag = a.flag;
   r.active = a.active;
   r.n_active = a.n_active;
-  r.tile_prefix = (path == NVFP4_PATH_GEMM) ? a.tile_prefix : nullptr;
-  r.tile_n = (path == NVFP4_PATH_GEMM) ? gemm_tile_n() : 0;
+  r.tile_prefix = a.tile_prefix;
+  r.tile_n = gemm_tile_n();
   if (int s = record(ev, 0, stream)) return s;
   if (int s = launch_route(r, stream, true)) return s;
   if (int s = record(ev, 1, stream)) return s;
-  if (path == NVFP4_PATH_GEMV) {
-    if (int s = launch_gemv_gateup(a, stream)) return s;
-    if (int s = record(ev, 2, stream)) return s;
-    if (int s = launch_gemv_down(a, stream)) return s;
-  } else {
-    if (int s = launch_gemm_gateup(a, stream)) return s;
-    if (int s = record(ev, 2, stream)) return s;
-    if (int s = launch_gemm_down(a, stream)) return s;
-  }
+  if (int s = launch_gemm_gateup(a, stream)) return s;
+  if (int s = record(ev, 2, stream)) return s;
+  if (int s = launch_gemm_down(a, stream)) return s;
   if (int s = record(ev, 3, stream)) return s;
   if (int s = launch_combine(a, stream)) return s;
   return record(ev, 4, stream);

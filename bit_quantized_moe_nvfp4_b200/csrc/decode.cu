@@ -1,229 +1,930 @@
-// decode.cu -- memory-bound GEMV path of the NVFP4 MoE layer (small token counts).
+// decode.cu -- memory-bound GEMV path of the NVFP4 MoE layer (few tokens per expert).
 //
-// Page "GLM-5-NVFP4-MTP", "Model Description": experts are NVFP4 (4-bit values, one FP8
-// scale per 16 elements), 8 of 256 active per token.  With few tokens per expert the layer
-// is a stream of packed expert bytes, so these kernels read every needed weight byte once
-// with 16-byte loads, decode E2M1 / E4M3 in registers with the hardware converts, and
-// accumulate in fp32 (packed FFMA2).  Each warp owns a contiguous range of equal-sized
-// work units (one gate/up row pair, or one or two down rows, of one active expert), so
-// the bytes are spread evenly over all warps of a persistent grid.
+// Page "GLM-5-NVFP4-MTP", "Model Description": the experts are NVFP4 (4-bit values with one
+// FP8 scale per 16 elements), 8 of 256 active per token.  With few tokens per expert the
+// layer is a stream of packed expert bytes, so two kernels read every needed weight byte
+// exactly once:
 //
-//   gate/up: a_j = g_gu * sum_h W[j,h] x[h] for the gate row j and the up row I+j together,
-//            then h_j = bf16(silu(gate) * up)  (SwiGLU fused, both rows in one warp)
-//   down:    y[r, n] = w[r] * g_dn * sum_i W[n,i] h[r,i]   for the expert's rows r
-// The combine over the K slots of a token runs afterwards (combine.cu).
+//   gemv_gateup: a_j = g_gu * (W_gu[j] . x) for the gate row j and the up row I+j of each
+//                active expert, then h_j = bf16(silu(gate) * up)        (SwiGLU fused)
+//   gemv_down:   y_k = g_dn * (W_dn . h_k) for every routed pair, then the top-k weighted
+//                combine out[t] = bf16(sum_k w[t,k] y_k) in ascending k    (combine fused)
+//
+// Each CTA routes the tokens itself (histogram of the ids, exclusive scan, stable ranks) so
+// no separate routing launch is needed.  One producer warp streams the CTA's contiguous
+// share of expert rows into a shared-memory ring with 1-D bulk copies (cp.async.bulk,
+// completion counted on mbarriers); the consumer warps split the reduction dimension so
+// each lane owns a fixed slice of the activations, kept in registers as f16 with an exact
+// per-token power-of-two scale.  Lanes decode E2M1 pairs and E4M3 scales with the hardware
+// converts and accumulate with mixed-precision fma.rn.f32.f16 (f16 x f16 products are exact,
+// sums are fp32); partial sums are combined across lanes by recursive-halving shuffles and
+// across warps through shared memory.
+//
+// Activation scaling: x_t is multiplied by 2^p_t with p_t = 14 - floor(log2 max|x_t|) and
+// rounded to f16.  bf16 has 8 significant bits and f16 11, so this is exact for every
+// element above 2^-31 * max|x_t| (smaller ones lose bits below f16's subnormal grid); the
+// dot products are rescaled by 2^-p_t in fp32.
 #include "moe.cuh"
+#include "pipeline.cuh"
 
 namespace nvfp4 {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+// Stage geometry (compile-time tunables; the defaults are the measured best on B200).
+#ifndef NVFP4_GEMV_STAGES
+#define NVFP4_GEMV_STAGES 2
+#endif
+#ifndef NVFP4_GEMV_PAIRS
+#define NVFP4_GEMV_PAIRS 4
+#endif
+#ifndef NVFP4_GEMV_DOWN_ROWS
+#define NVFP4_GEMV_DOWN_ROWS 8
+#endif
+#ifndef NVFP4_GEMV_CTAS_PER_SM
+#define NVFP4_GEMV_CTAS_PER_SM 3
+#endif
+#ifndef NVFP4_GEMV_DOWN_CTAS_PER_SM
+#define NVFP4_GEMV_DOWN_CTAS_PER_SM 4
+#endif
+constexpr int kStages = NVFP4_GEMV_STAGES;       // shared-memory ring depth
+constexpr int kPairs = NVFP4_GEMV_PAIRS;         // gate/up row pairs per stage
+constexpr int kDownRows = NVFP4_GEMV_DOWN_ROWS;  // rows per stage (down kernel)
+constexpr int kMaxConsumerWarps = 6;
+constexpr int64_t kGemvMaxPairs = 1024;  // T*K handled by the GEMV path
 
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
-// 8 E2M1 codes (one 32-bit word) -> 4 float2 (elements 2p, 2p+1), exact.
-__device__ __forceinline__ void decode8(uint32_t word, float2 (&q)[4]) {
-  uint32_t h[4];
-  e2m1x8_to_f16x2x4(word, h);
+// ------------------------------------------------------------------ small helpers
+__device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
-  for (int p = 0; p < 4; ++p) q[p] = __half22float2(*reinterpret_cast<__half2 *>(&h[p]));
-}
-
-// 8 bf16 (one uint4) -> 4 float2, exact.
-__device__ __forceinline__ void bf16x8(uint4 v, float2 (&f)[4]) {
-  f[0] = make_float2(bf16_lo(v.x), bf16_hi(v.x));
-  f[1] = make_float2(bf16_lo(v.y), bf16_hi(v.y));
-  f[2] = make_float2(bf16_lo(v.z), bf16_hi(v.z));
-  f[3] = make_float2(bf16_lo(v.w), bf16_hi(v.w));
-}
-
-// Dot product of one 32-element chunk (16 packed bytes, 2 block scales) with 32 fp32
-// activations given as 4 uint4 of bf16; returns acc + s0 * dot(block 0) + s1 * dot(block 1).
-__device__ __forceinline__ float2 chunk_dot(uint4 q, float s0, float s1, const uint4 (&xv)[4],
-                                            float2 acc) {
-  const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    float2 part = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      float2 qf[4], xf[4];
-      decode8(words[2 * b + w], qf);
-      bf16x8(xv[2 * b + w], xf);
-#pragma unroll
-      for (int p = 0; p < 4; ++p) part = ffma2(qf[p], xf[p], part);
-    }
-    const float s = b ? s1 : s0;
-    acc = ffma2(part, make_float2(s, s), acc);
-  }
-  return acc;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
 }
 
-__device__ __forceinline__ void load_x_chunk(const __nv_bfloat16 *row, int c, uint4 (&xv)[4]) {
-  const uint4 *p = reinterpret_cast<const uint4 *>(row + 32 * c);
+// Sum each of M per-lane values over the warp (M a power of two <= 32) by recursive
+// halving: afterwards lane l holds the total of value index (l >> (5 - log2 M)).
+template <int M>
+__device__ __forceinline__ float warp_reduce_many(float (&v)[M], int lane) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) xv[i] = __ldg(p + i);
+  for (int width = M; width > 1; width >>= 1) {
+    const int d = (16 * width) / M;
+    const bool upper = (lane & d) != 0;
+#pragma unroll
+    for (int i = 0; i < width / 2; ++i) {
+      const float send = upper ? v[i] : v[i + width / 2];
+      const float keep = upper ? v[i + width / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, d);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int d = 16 / M; d >= 1; d >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, d);
+  return r;
 }
 
-__device__ __forceinline__ void scales2(const uint8_t *srow, int c, float &s0, float &s1) {
-  const uint32_t two = __ldg(reinterpret_cast<const unsigned short *>(srow) + c);
-  const uint32_t h = e4m3x2_to_f16x2(two);
-  s0 = f16_lo(h);
-  s1 = f16_hi(h);
+template <int M>
+struct Log2 {
+  static constexpr int value = (M <= 1) ? 0 : 1 + Log2<M / 2>::value;
+};
+template <>
+struct Log2<1> {
+  static constexpr int value = 0;
+};
+
+// v[i] for a runtime i < N without dynamic register indexing.
+template <int N, typename V>
+__device__ __forceinline__ V pick(const V (&v)[N], int i) {
+  V r = v[0];
+#pragma unroll
+  for (int k = 1; k < N; ++k)
+    if (i == k) r = v[k];
+  return r;
 }
 
-// ------------------------------------------------------------------ gate/up + SwiGLU
+// Power of two 2^p as fp32, p in [-126, 127].
+__device__ __forceinline__ float exp2i(int p) { return __uint_as_float((uint32_t)(p + 127) << 23); }
+
+// Scale exponent for a token whose largest magnitude is m: m * 2^p lands in [2^14, 2^15).
+__device__ __forceinline__ int prescale_exponent(float m) {
+  if (!(m > 0.0f)) return 0;
+  const int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 127;  // floor(log2 m) for normals
+  int p = 14 - e;
+  p = max(-100, min(100, p));
+  return p;
+}
+
+// 2 x f32 -> f16x2 (round to nearest even)
+__device__ __forceinline__ uint32_t f16x2_rn(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// acc += lo(q) * lo(x) and acc2 += hi(q) * hi(x), f16 operands, fp32 accumulate.
+__device__ __forceinline__ void fma_f16x2_f32(uint32_t q, uint32_t x, float &acc, float &acc2) {
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\t"
+      "mov.b32 {a0, a1}, %2;\n\tmov.b32 {b0, b1}, %3;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %0;\n\tfma.rn.f32.f16 %1, a1, b1, %1;\n\t}"
+      : "+f"(acc), "+f"(acc2)
+      : "r"(q), "r"(x));
+}
+
+// Dot of 16 E2M1 codes (two words) with 16 f16 activations (8 f16x2 registers), fp32.
+__device__ __forceinline__ float dot16(uint32_t w0, uint32_t w1, const uint32_t *xh) {
+  uint32_t q[8];
+  e2m1x8_to_f16x2x4(w0, *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
+  e2m1x8_to_f16x2x4(w1, *reinterpret_cast<uint32_t(*)[4]>(&q[4]));
+  float a = 0.f, b = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) fma_f16x2_f32(q[i], xh[i], a, b);
+  return a + b;
+}
+
+// Bulk copies move 16-byte-aligned runs of a multiple of 16 bytes.  A run of scale rows
+// (rows * cols/16 bytes) need not be aligned, so the aligned superset is copied instead:
+// it stays inside the expert's own scale block, whose size rows_total * cols/16 is a
+// multiple of 16 (rows and cols are multiples of 64).  Returns the bytes issued; the
+// wanted data starts `lead` = begin % 16 bytes into dst.
+__device__ __forceinline__ uint32_t bulk_g2s_span(void *dst, const uint8_t *block, int64_t begin,
+                                                  int64_t len, uint64_t *bar) {
+  const int64_t b = begin & ~int64_t(15);
+  const int64_t e = (begin + len + 15) & ~int64_t(15);
+  bulk_g2s(dst, block + b, (uint32_t)(e - b), bar);
+  return (uint32_t)(e - b);
+}
+
+__host__ __device__ __forceinline__ uint32_t span_bytes(int64_t len) { return (uint32_t)len + 32; }
+
+// ------------------------------------------------------------------ in-CTA routing
+// Shared-memory routing tables of one CTA.
+struct CtaRoute {
+  int *ids;      // [n]  expert id of pair p (copy of topk_ids)
+  int *act_e;    // [min(E, n)]  active experts, ascending
+  int *act_off;  // [min(E, n) + 1]  first slot of each active expert
+  int *n_act;    // [1]
+};
+
+// All threads of the CTA: copy the ids, count pairs per expert (hist[E] is scratch), and
+// list the active experts with the exclusive prefix of their counts.  hist[e] ends up as
+// the active index of expert e (-1 if none).  Returns true if some id is out of range.
+__device__ bool cta_route(const int32_t *g_ids, int n, int E, CtaRoute r, int *hist) {
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31;
+  if (tid == 0) s_bad = 0;
+  for (int e = tid; e < E; e += nth) hist[e] = 0;
+  // ids are read past L1: they may have been written by the kernel this one follows
+  for (int p = tid; p < n; p += nth) r.ids[p] = __ldcg(g_ids + p);
+  __syncthreads();
+  bool bad = false;
+  for (int p = tid; p < n; p += nth) {
+    const int v = r.ids[p];
+    if (v >= 0 && v < E)
+      atomicAdd(&hist[v], 1);
+    else
+      bad = true;
+  }
+  if (bad) s_bad = 1;
+  __syncthreads();
+  if (tid < 32) {
+    const int per = (E + 31) / 32;
+    const int e0 = lane * per, e1 = min(E, e0 + per);
+    int run = 0, act = 0;
+    for (int e = e0; e < e1; ++e) {
+      run += hist[e];
+      act += hist[e] > 0;
+    }
+    int incl = run, iact = act;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      const int w = __shfl_up_sync(0xFFFFFFFFu, iact, o);
+      if (lane >= o) {
+        incl += v;
+        iact += w;
+      }
+    }
+    int pos = incl - run, apos = iact - act;
+    for (int e = e0; e < e1; ++e) {
+      const int c = hist[e];
+      if (c > 0) {
+        r.act_e[apos] = e;
+        r.act_off[apos] = pos;
+        hist[e] = apos;
+        ++apos;
+      } else {
+        hist[e] = -1;
+      }
+      pos += c;
+    }
+    if (lane == 31) {
+      r.act_off[apos] = pos;
+      *r.n_act = apos;
+    }
+  }
+  __syncthreads();
+  return s_bad != 0;
+}
+
+// The pairs p (ascending) routed to expert e with rank in [first, first + NT): lane i < NT
+// of the calling warp receives the i-th one (-1 past the end).
 template <int NT>
-__global__ void __launch_bounds__(kThreads) gemv_gateup_kernel(MoeArgs a) {
-  pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t warps_total = (int64_t)gridDim.x * kWarps;
-  const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int64_t I = a.I, H = a.H, K = a.K;
-  const int64_t units = (int64_t)(*a.n_active) * I;
-  const int64_t u0 = units * gw / warps_total, u1 = units * (gw + 1) / warps_total;
-  const int nchunks = (int)(H / 32);
+__device__ int pairs_of_expert(const int *ids, int n, int e, int first, int lane) {
+  int seen = 0, mine = -1;
+  for (int base = 0; base < n && seen < first + NT; base += 32) {
+    const int p = base + lane;
+    const bool m = p < n && ids[p] == e;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, m);
+    const int rank = seen + __popc(bal & ((1u << lane) - 1u));
+    // hand pair p to lane (rank - first)
+    const int want = lane + first;   // the rank lane `lane` is looking for
+#pragma unroll 1
+    for (unsigned b = bal; b; b &= b - 1) {
+      const int src = __ffs(b) - 1;
+      const int rk = __shfl_sync(0xFFFFFFFFu, rank, src);
+      if (rk == want) mine = base + src;
+    }
+    seen += __popc(bal);
+  }
+  return lane < NT ? mine : -1;
+}
 
-  for (int64_t u = u0; u < u1; ++u) {
-    const int e = a.active[u / I];
+// Slot (row of h) of every pair: slot = first slot of its expert + stable rank; -1 for an
+// out-of-range id.  One warp; run[] is scratch of n_act ints.
+__device__ void warp_slots(const int *ids, int n, int E, const int *act_index, const int *act_off,
+                           int n_act, int *run, int *slot, int lane) {
+  for (int a = lane; a < n_act; a += 32) run[a] = act_off[a];
+  __syncwarp();
+  for (int base = 0; base < n; base += 32) {
+    const int p = base + lane;
+    const int v = p < n ? ids[p] : -1;
+    const bool valid = v >= 0 && v < E;
+    const unsigned key = valid ? (unsigned)v : 0x80000000u | (unsigned)lane;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int ai = valid ? act_index[v] : -1;
+    const int s = valid ? run[ai] + rank : -1;
+    __syncwarp();
+    if (valid && rank == 0) run[ai] += __popc(peers);
+    __syncwarp();
+    if (p < n) slot[p] = s;
+  }
+}
+
+// Load one activation slice (32 bf16 at src) for a lane, return its max |x| (fp32).
+__device__ __forceinline__ float load_bf16x32(const __nv_bfloat16 *src, uint4 (&v)[4]) {
+  const uint4 *p = reinterpret_cast<const uint4 *>(src);
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[i] = __ldcg(p + i);
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[k])), fabsf(bf16_hi(w[k]))));
+  }
+  return m;
+}
+
+// 32 bf16 -> 16 f16x2 after scaling by s (exact power of two)
+__device__ __forceinline__ void to_f16x32(const uint4 (&v)[4], float s, uint32_t *xh) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) xh[4 * i + k] = f16x2_rn(bf16_lo(w[k]) * s, bf16_hi(w[k]) * s);
+  }
+}
+
+// Shared memory carve-up common to both kernels (offsets in bytes from the dynamic base).
+// Barriers: full[S] / empty[S] for the stage ring, rfull[R] / rfree[R] for the ring of
+// reduction slots that carries partial sums from the consumer warps to the finalizer warp.
+constexpr int kRedSlots = 4;
+
+struct Smem {
+  uint32_t bars, stages, red, smax, ids, act_e, act_off, misc, slot, run, hist, yk, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Floats per reduction slot: CW * red_vals partial sums + 2 * 4 per-token extras.
+__host__ __device__ inline int red_slot_floats(int cw, int red_vals) { return cw * red_vals + 8; }
+
+__host__ __device__ inline Smem smem_layout(int S, uint32_t stage_bytes, int cw, int red_vals,
+                                            int n, int E, int yk_floats) {
+  Smem s;
+  uint32_t o = 0;
+  s.bars = o;
+  o += 8 * (2 * S + 2 * kRedSlots);
+  o = align_up(o, 128);
+  s.stages = o;
+  o += stage_bytes * S;
+  s.red = o;
+  o += 4 * kRedSlots * red_slot_floats(cw, red_vals);
+  s.smax = o;
+  o += 4 * cw * 4;
+  s.ids = o;
+  o += 4 * n;
+  const int na = min(E, n);
+  s.act_e = o;
+  o += 4 * na;
+  s.act_off = o;
+  o += 4 * (na + 1);
+  s.misc = o;
+  o += 16;
+  s.slot = o;
+  o += 4 * n;
+  s.run = o;
+  o += 4 * na;
+  s.hist = o;
+  o += 4 * E;
+  o = align_up(o, 16);
+  s.yk = o;
+  o += 4 * yk_floats;
+  s.total = align_up(o, 128);
+  return s;
+}
+
+// Wait on an mbarrier phase with the whole warp agreeing on the outcome.  Once any wait of
+// the CTA has given up (abort set), later waits are skipped and report failure, so every
+// role still runs its loops to the end (arrivals included) without blocking.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *abort,
+                                          int32_t *flag) {
+  bool ok = false;
+  if (!*(volatile int *)abort) ok = mbar_wait(bar, parity);
+  ok = __all_sync(0xFFFFFFFFu, ok);
+  if (!ok && !*(volatile int *)abort && (threadIdx.x & 31) == 0) {
+    *(volatile int *)abort = 1;
+    report_timeout(flag);
+  }
+  return ok;
+}
+
+// ================================================================== gate/up + SwiGLU
+// blockDim = 32 * (CW + 2): warp 0 produces (bulk copies), warps 1..CW compute, warp CW+1
+// finalizes.  Each computing lane owns 32 consecutive elements (16 packed bytes, 2 block
+// scales) of every row; a stage holds P gate rows and the P matching up rows of one expert.
+template <int NT, int P, int S>
+__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 3 : 1)
+    gemv_gateup_kernel(MoeArgs a, uint32_t stage_bytes) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_abort;
+  const int CW = blockDim.x / 32 - 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t H = a.H, I = a.I, K = a.K;
+  const int n = (int)(a.T * K);
+  const int E = (int)a.E;
+  constexpr int RV = 2 * P * NT;   // values reduced per stage per lane
+  const int RS = red_slot_floats(CW, RV);
+  const Smem L = smem_layout(S, stage_bytes, CW, RV, n, E, 0);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
+  uint64_t *empty = full + S;
+  uint64_t *rfull = empty + S;
+  uint64_t *rfree = rfull + kRedSlots;
+  unsigned char *stage_base = smem + L.stages;
+  float *red = reinterpret_cast<float *>(smem + L.red);
+  float *smax = reinterpret_cast<float *>(smem + L.smax);
+  CtaRoute R{reinterpret_cast<int *>(smem + L.ids), reinterpret_cast<int *>(smem + L.act_e),
+             reinterpret_cast<int *>(smem + L.act_off), reinterpret_cast<int *>(smem + L.misc)};
+  int *hist = reinterpret_cast<int *>(smem + L.hist);
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], CW);
+    }
+    for (int s = 0; s < kRedSlots; ++s) {
+      mbar_init(&rfull[s], CW);
+      mbar_init(&rfree[s], 1);
+    }
+    mbar_init_fence();
+  }
+  pdl_wait();  // x and the ids come from earlier kernels
+  const bool bad = cta_route(a.ids, n, E, R, hist);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.flag) *a.flag = bad ? kFlagBadId : 0;
+  pdl_launch_dependents();  // the down kernel may start routing and prefetching
+
+  const int n_act = *R.n_act;
+  const int64_t units = (int64_t)n_act * I;
+  const int64_t U0 = units * blockIdx.x / gridDim.x, U1 = units * (blockIdx.x + 1) / gridDim.x;
+  const uint32_t rowb = (uint32_t)(H / 2), sclb = (uint32_t)(H / 16);
+  const uint32_t span_stride = span_bytes(P * sclb);
+
+  if (warp == 0) {
+    // ------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      for (int64_t u = U0; u < U1; ++s) {
+        const int ai = (int)(u / I);
+        const int64_t j = u % I;
+        const int np = (int)min64(min64(P, I - j), U1 - u);
+        const int e = R.act_e[ai];
+        const int idx = s % S;
+        if (s >= S && (*(volatile int *)&s_abort || !mbar_wait(&empty[idx], ((s / S) - 1) & 1))) {
+          if (!*(volatile int *)&s_abort) report_timeout(a.flag);
+          *(volatile int *)&s_abort = 1;
+          break;
+        }
+        unsigned char *st = stage_base + (size_t)idx * stage_bytes;
+        const int64_t rg = (int64_t)e * 2 * I + j;   // first gate row
+        const int64_t ru = rg + I;                   // first up row
+        const uint8_t *sblock = a.s_gu + (int64_t)e * 2 * I * sclb;
+        const int64_t lg = j * sclb, lu = (I + j) * sclb;   // offsets inside the block
+        const uint32_t span_g = (uint32_t)(((lg + np * sclb + 15) & ~15ll) - (lg & ~15ll));
+        const uint32_t span_u = (uint32_t)(((lu + np * sclb + 15) & ~15ll) - (lu & ~15ll));
+        mbar_arrive_expect_tx(&full[idx], 2u * np * rowb + span_g + span_u);
+        bulk_g2s(st, a.w_gu + rg * rowb, np * rowb, &full[idx]);
+        bulk_g2s(st + P * rowb, a.w_gu + ru * rowb, np * rowb, &full[idx]);
+        unsigned char *sc = st + 2 * P * rowb;
+        bulk_g2s_span(sc, sblock, lg, np * sclb, &full[idx]);
+        bulk_g2s_span(sc + span_stride, sblock, lu, np * sclb, &full[idx]);
+        u += np;
+      }
+      // do not leave while copies into this CTA's shared memory may still be in flight
+      const int issued = s;
+      for (int t = max(0, issued - S); t < issued; ++t)
+        if (!mbar_wait(&full[t % S], (t / S) & 1)) report_timeout(a.flag);
+    }
+    return;
+  }
+
+  if (warp == CW + 1) {
+    // ------------------------------------------------ finalizer
+    int it = 0, cur_a = -1, slot0 = 0, cnt = 0;
+    float g = 0.f;
+    for (int64_t u = U0; u < U1;) {
+      const int ai = (int)(u / I);
+      const int64_t j = u % I;
+      const int np = (int)min64(min64(P, I - j), U1 - u);
+      if (ai != cur_a) {
+        cur_a = ai;
+        slot0 = R.act_off[ai];
+        cnt = R.act_off[ai + 1] - slot0;
+        g = __ldg(a.g_gu + R.act_e[ai]);
+      }
+      for (int grp = 0; grp * NT < cnt; ++grp, ++it) {
+        const int nt = min(NT, cnt - grp * NT);
+        const int sl = it % kRedSlots;
+        const bool ok = warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag);
+        const float *rb = red + (size_t)sl * RS;
+        if (ok && lane < np * nt) {
+          const int pp = lane / nt, i = lane % nt;
+          float gs = 0.f, us = 0.f;
+          for (int w = 0; w < CW; ++w) {
+            gs += rb[w * RV + pp * NT + i];
+            us += rb[w * RV + (P + pp) * NT + i];
+          }
+          const float ps = rb[CW * RV + i];
+          const float gate = gs * g * ps;
+          const float up = us * g * ps;
+          const int slot = slot0 + grp * NT + i;
+          a.h[(int64_t)slot * I + j + pp] = __float2bfloat16_rn(silu_f32(gate) * up);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfree[sl]);
+      }
+      u += np;
+    }
+    return;
+  }
+
+  // ------------------------------------------------ compute warps
+  const int cw = warp - 1;                       // compute warp index
+  const int chunk = cw * 32 + lane;              // 32-element chunk owned by this lane
+  const bool owns = chunk < (int)(H / 32);
+  const int nthreads_c = CW * 32;
+  uint32_t xh[NT][16];
+  float pscale[NT];                              // 2^-p per token of the current group
+  int loaded_tok[NT];                            // tokens whose activations are in xh
+#pragma unroll
+  for (int i = 0; i < NT; ++i) loaded_tok[i] = -1;
+  int cur_a = -1, ngroups = 0, cnt = 0;
+  int s = 0, it = 0;
+  for (int64_t u = U0; u < U1; ++s) {
+    const int ai = (int)(u / I);
     const int64_t j = u % I;
-    const int off = a.offsets[e], cnt = a.counts[e];
-    const uint8_t *pg = a.w_gu + ((int64_t)e * 2 * I + j) * (H / 2);
-    const uint8_t *pu = pg + I * (H / 2);
-    const uint8_t *sg = a.s_gu + ((int64_t)e * 2 * I + j) * (H / 16);
-    const uint8_t *su = sg + I * (H / 16);
-    const float g = __ldg(a.g_gu + e);
-    for (int t0 = 0; t0 < cnt; t0 += NT) {
-      const int nt = min(NT, cnt - t0);
-      const __nv_bfloat16 *xr[NT];
-#pragma unroll
-      for (int i = 0; i < NT; ++i)
-        xr[i] = a.x + (int64_t)(a.perm[off + t0 + min(i, nt - 1)] / K) * H;
-      float2 ag[NT], au[NT];
-#pragma unroll
-      for (int i = 0; i < NT; ++i) ag[i] = au[i] = make_float2(0.f, 0.f);
-#pragma unroll 2
-      for (int c = lane; c < nchunks; c += 32) {
-        const uint4 qg = ldg_stream(pg + 16 * c);
-        const uint4 qu = ldg_stream(pu + 16 * c);
-        float sg0, sg1, su0, su1;
-        scales2(sg, c, sg0, sg1);
-        scales2(su, c, su0, su1);
+    const int np = (int)min64(min64(P, I - j), U1 - u);
+    const int idx = s % S;
+    const bool new_expert = ai != cur_a;
+    if (new_expert) {
+      cur_a = ai;
+      cnt = R.act_off[ai + 1] - R.act_off[ai];
+      ngroups = (cnt + NT - 1) / NT;
+    }
+    const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
+    const unsigned char *st = stage_base + (size_t)idx * stage_bytes;
+    const int64_t offg = j * sclb, offu = (I + j) * sclb;
+    const unsigned char *spg = st + 2 * P * rowb + (offg & 15);
+    const unsigned char *spu = st + 2 * P * rowb + span_stride + (offu & 15);
+    for (int grp = 0; grp < ngroups; ++grp, ++it) {
+      const int nt = min(NT, cnt - grp * NT);
+      const bool last = grp == ngroups - 1;
+      // (re)load the activations of this token group when they are not in registers
+      bool reload = false;
+      int tok[NT];
+      if (ngroups > 1 || new_expert) {
+        // the same tokens as the ones in registers (always so for a single token) need no
+        // reload; the decision depends only on shared data, so all compute warps agree
+        const int pr = pairs_of_expert<NT>(R.ids, n, R.act_e[ai], grp * NT, lane);
 #pragma unroll
         for (int i = 0; i < NT; ++i) {
-          if (i < nt) {
-            uint4 xv[4];
-            load_x_chunk(xr[i], c, xv);
-            ag[i] = chunk_dot(qg, sg0, sg1, xv, ag[i]);
-            au[i] = chunk_dot(qu, su0, su1, xv, au[i]);
+          tok[i] = (int)(__shfl_sync(0xFFFFFFFFu, pr, min(i, nt - 1)) / K);
+          reload |= tok[i] != loaded_tok[i];
+        }
+      }
+      if (reload) {
+        const __nv_bfloat16 *xr[NT];
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+          loaded_tok[i] = tok[i];
+          xr[i] = a.x + (int64_t)tok[i] * H + chunk * 32;
+        }
+        // pass 1: largest magnitude of each token (over all compute warps)
+        float m[NT];
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+          uint4 v[4];
+          m[i] = warp_max(owns ? load_bf16x32(xr[i], v) : 0.f);
+        }
+        if (lane == 0)
+#pragma unroll
+          for (int i = 0; i < NT; ++i) smax[cw * 4 + i] = m[i];
+        named_sync(1, nthreads_c);
+        // pass 2: scale by 2^p and round to f16 (the reload hits L1/L2)
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+          float mm = 0.f;
+          for (int w = 0; w < CW; ++w) mm = fmaxf(mm, smax[w * 4 + i]);
+          const int p = prescale_exponent(mm);
+          pscale[i] = exp2i(-p);
+          if (owns) {
+            uint4 v[4];
+            load_bf16x32(xr[i], v);
+            to_f16x32(v, exp2i(p), xh[i]);
+          }
+        }
+        named_sync(1, nthreads_c);   // smax is rewritten by the next load
+      }
+      // partial dot products of all 2P rows (rows past np hold stale data and are ignored)
+      float flat[RV];
+#pragma unroll
+      for (int v = 0; v < RV; ++v) flat[v] = 0.f;
+      if (owns && have) {
+#pragma unroll
+        for (int r = 0; r < 2 * P; ++r) {
+          const uint4 q = *reinterpret_cast<const uint4 *>(st + (size_t)r * rowb + chunk * 16);
+          const unsigned char *sp = (r < P) ? spg : spu;
+          const uint32_t sc2 = *reinterpret_cast<const unsigned short *>(
+              sp + (size_t)(r % P) * sclb + chunk * 2);
+          const uint32_t s16 = e4m3x2_to_f16x2(sc2);
+          const float s0 = f16_lo(s16), s1 = f16_hi(s16);
+#pragma unroll
+          for (int i = 0; i < NT; ++i) {
+            const float d0 = dot16(q.x, q.y, &xh[i][0]);
+            const float d1 = dot16(q.z, q.w, &xh[i][8]);
+            flat[r * NT + i] = fmaf(d1, s1, d0 * s0);
           }
         }
       }
+      if (last) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[idx]);   // this warp is done reading the stage
+      }
+      const float tot = warp_reduce_many<RV>(flat, lane);
+      constexpr int SH = 5 - Log2<RV>::value;
+      const int sl = it % kRedSlots;
+      if (it >= kRedSlots) warp_wait(&rfree[sl], ((it / kRedSlots) - 1) & 1, &s_abort, a.flag);
+      float *rb = red + (size_t)sl * RS;
+      if ((lane & ((1 << SH) - 1)) == 0) rb[cw * RV + (lane >> SH)] = tot;
+      if (cw == 0 && lane < NT) rb[CW * RV + lane] = pick<NT>(pscale, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfull[sl]);
+    }
+    u += np;
+  }
+}
+
+// ================================================================== down + combine
+// CTA c owns output rows [n0, n0 + nb) for every active expert.  Warp 0 produces, warps
+// 1..CW compute with lanes owning 16 consecutive elements (8 packed bytes, 1 block scale),
+// warp CW+1 finalizes.  Per-pair results stay in shared memory (yk) and are combined in
+// ascending k at the end.
+template <int NT, int RD, int S>
+__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
+    gemv_down_kernel(MoeArgs a, uint32_t stage_bytes, int nb) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_abort;
+  const int CW = blockDim.x / 32 - 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t H = a.H, I = a.I, K = a.K, T = a.T;
+  const int n = (int)(T * K);
+  const int E = (int)a.E;
+  constexpr int RV = RD * NT;
+  const int RS = red_slot_floats(CW, RV);
+  const Smem L = smem_layout(S, stage_bytes, CW, RV, n, E, n * nb);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
+  uint64_t *empty = full + S;
+  uint64_t *rfull = empty + S;
+  uint64_t *rfree = rfull + kRedSlots;
+  unsigned char *stage_base = smem + L.stages;
+  float *red = reinterpret_cast<float *>(smem + L.red);
+  float *smax = reinterpret_cast<float *>(smem + L.smax);
+  CtaRoute R{reinterpret_cast<int *>(smem + L.ids), reinterpret_cast<int *>(smem + L.act_e),
+             reinterpret_cast<int *>(smem + L.act_off), reinterpret_cast<int *>(smem + L.misc)};
+  int *hist = reinterpret_cast<int *>(smem + L.hist);
+  int *slot_of = reinterpret_cast<int *>(smem + L.slot);
+  int *run = reinterpret_cast<int *>(smem + L.run);
+  float *yk = reinterpret_cast<float *>(smem + L.yk);
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], CW);
+    }
+    for (int s = 0; s < kRedSlots; ++s) {
+      mbar_init(&rfull[s], CW);
+      mbar_init(&rfree[s], 1);
+    }
+    mbar_init_fence();
+  }
+  // The ids were complete before the gate/up kernel let this grid start; reading them
+  // (and the weights) before griddepcontrol.wait overlaps this prologue with its tail.
+  cta_route(a.ids, n, E, R, hist);
+  const int n_act = *R.n_act;
+  if (warp == 1) warp_slots(R.ids, n, E, hist, R.act_off, n_act, run, slot_of, lane);
+  __syncthreads();
+
+  const int n0 = blockIdx.x * nb;
+  const int n1 = min((int)H, n0 + nb);
+  const uint32_t rowb = (uint32_t)(I / 2), sclb = (uint32_t)(I / 16);
+  const int rows_per_expert = n1 > n0 ? (n1 - n0) : 0;
+  const int chunks_per_expert = (rows_per_expert + RD - 1) / RD;
+  const int n_stages = n_act * chunks_per_expert;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      for (; s < n_stages; ++s) {
+        const int ai = s / chunks_per_expert;
+        const int r0 = n0 + (s % chunks_per_expert) * RD;
+        const int nr = min(RD, n1 - r0);
+        const int e = R.act_e[ai];
+        const int idx = s % S;
+        if (s >= S && (*(volatile int *)&s_abort || !mbar_wait(&empty[idx], ((s / S) - 1) & 1))) {
+          if (!*(volatile int *)&s_abort) report_timeout(a.flag);
+          *(volatile int *)&s_abort = 1;
+          break;
+        }
+        unsigned char *st = stage_base + (size_t)idx * stage_bytes;
+        const int64_t row = (int64_t)e * H + r0;
+        const int64_t ls = (int64_t)r0 * sclb;
+        const uint32_t span = (uint32_t)(((ls + nr * sclb + 15) & ~15ll) - (ls & ~15ll));
+        mbar_arrive_expect_tx(&full[idx], (uint32_t)nr * rowb + span);
+        bulk_g2s(st, a.w_dn + row * rowb, nr * rowb, &full[idx]);
+        bulk_g2s_span(st + RD * rowb, a.s_dn + (int64_t)e * H * sclb, ls, nr * sclb, &full[idx]);
+      }
+      const int issued = s;
+      for (int t = max(0, issued - S); t < issued; ++t)
+        if (!mbar_wait(&full[t % S], (t / S) & 1)) report_timeout(a.flag);
+    }
+    return;
+  }
+
+  const int nthreads_cf = (CW + 1) * 32;   // compute + finalizer threads (combine)
+  if (warp == CW + 1) {
+    // ------------------------------------------------ finalizer
+    int it = 0;
+    for (int s = 0; s < n_stages; ++s) {
+      const int ai = s / chunks_per_expert;
+      const int r0 = n0 + (s % chunks_per_expert) * RD;
+      const int nr = min(RD, n1 - r0);
+      const int slot0 = R.act_off[ai];
+      const int cnt = R.act_off[ai + 1] - slot0;
+      const float g = __ldg(a.g_dn + R.act_e[ai]);
+      for (int grp = 0; grp * NT < cnt; ++grp, ++it) {
+        const int nt = min(NT, cnt - grp * NT);
+        const int sl = it % kRedSlots;
+        const bool ok = warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag);
+        const float *rb = red + (size_t)sl * RS;
+        if (ok && lane < nr * nt) {
+          const int rr = lane / nt, i = lane % nt;
+          float sum = 0.f;
+          for (int w = 0; w < CW; ++w) sum += rb[w * RV + rr * NT + i];
+          const float ps = rb[CW * RV + i];
+          const int pair = __float_as_int(rb[CW * RV + 4 + i]);
+          const int slot = slot0 + grp * NT + i;
+          yk[(size_t)slot * nb + (r0 - n0) + rr] = sum * g * ps * __ldg(a.w + pair);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfree[sl]);
+      }
+    }
+  } else {
+    // ------------------------------------------------ compute warps
+    pdl_wait();   // h is written by the gate/up kernel
+    pdl_launch_dependents();
+    const int cw = warp - 1;
+    const int nthreads_c = CW * 32;
+    const int chunk = cw * 32 + lane;              // 16-element chunk owned by this lane
+    const bool owns = chunk < (int)(I / 16);
+    uint32_t xh[NT][8];
+    float pscale[NT];
+    int pair_of[NT];
+    int cur_a = -1, ngroups = 0, cnt = 0, slot0 = 0;
+    int it = 0;
+    for (int s = 0; s < n_stages; ++s) {
+      const int ai = s / chunks_per_expert;
+      const int r0 = n0 + (s % chunks_per_expert) * RD;
+      const int idx = s % S;
+      const bool new_expert = ai != cur_a;
+      if (new_expert) {
+        cur_a = ai;
+        slot0 = R.act_off[ai];
+        cnt = R.act_off[ai + 1] - slot0;
+        ngroups = (cnt + NT - 1) / NT;
+      }
+      const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
+      const unsigned char *st = stage_base + (size_t)idx * stage_bytes;
+      const unsigned char *sbase = st + RD * rowb + (((int64_t)r0 * sclb) & 15);
+      for (int grp = 0; grp < ngroups; ++grp, ++it) {
+        const int nt = min(NT, cnt - grp * NT);
+        const bool last = grp == ngroups - 1;
+        if (ngroups > 1 || new_expert) {
+          // h rows of this group's slots (slot = slot0 + grp*NT + i), scaled to f16
+          const int pr = pairs_of_expert<NT>(R.ids, n, R.act_e[ai], grp * NT, lane);
+          const uint4 *hp[NT];
+          float m[NT];
 #pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        if (i < nt) {
-          const float gate = warp_sum(ag[i].x + ag[i].y) * g;
-          const float up = warp_sum(au[i].x + au[i].y) * g;
-          if (lane == 0) {
-            const float hv = silu_f32(gate) * up;
-            a.h[(int64_t)(off + t0 + i) * I + j] = __float2bfloat16_rn(hv);
+          for (int i = 0; i < NT; ++i) {
+            pair_of[i] = __shfl_sync(0xFFFFFFFFu, pr, min(i, nt - 1));
+            const int slot = slot0 + grp * NT + min(i, nt - 1);
+            hp[i] = reinterpret_cast<const uint4 *>(a.h + (int64_t)slot * I + chunk * 16);
+            float mm = 0.f;
+            if (owns) {
+#pragma unroll
+              for (int k2 = 0; k2 < 2; ++k2) {
+                const uint4 v = __ldcg(hp[i] + k2);
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  mm = fmaxf(mm, fmaxf(fabsf(bf16_lo(w4[k])), fabsf(bf16_hi(w4[k]))));
+              }
+            }
+            m[i] = warp_max(mm);
+          }
+          if (lane == 0)
+#pragma unroll
+            for (int i = 0; i < NT; ++i) smax[cw * 4 + i] = m[i];
+          named_sync(1, nthreads_c);
+#pragma unroll
+          for (int i = 0; i < NT; ++i) {
+            float mm = 0.f;
+            for (int w = 0; w < CW; ++w) mm = fmaxf(mm, smax[w * 4 + i]);
+            const int p = prescale_exponent(mm);
+            pscale[i] = exp2i(-p);
+            if (owns) {
+              const float sp = exp2i(p);
+#pragma unroll
+              for (int k2 = 0; k2 < 2; ++k2) {
+                const uint4 v = __ldcg(hp[i] + k2);
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  xh[i][4 * k2 + k] = f16x2_rn(bf16_lo(w4[k]) * sp, bf16_hi(w4[k]) * sp);
+              }
+            }
+          }
+          named_sync(1, nthreads_c);
+        }
+        float flat[RV];
+#pragma unroll
+        for (int v = 0; v < RV; ++v) flat[v] = 0.f;
+        if (owns && have) {
+#pragma unroll
+          for (int r = 0; r < RD; ++r) {
+            const uint2 q = *reinterpret_cast<const uint2 *>(st + (size_t)r * rowb + chunk * 8);
+            const float sc = e4m3_to_f32(sbase[(size_t)r * sclb + chunk]);
+#pragma unroll
+            for (int i = 0; i < NT; ++i) flat[r * NT + i] = dot16(q.x, q.y, &xh[i][0]) * sc;
           }
         }
+        if (last) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[idx]);
+        }
+        const float tot = warp_reduce_many<RV>(flat, lane);
+        constexpr int SH = 5 - Log2<RV>::value;
+        const int sl = it % kRedSlots;
+        if (it >= kRedSlots) warp_wait(&rfree[sl], ((it / kRedSlots) - 1) & 1, &s_abort, a.flag);
+        float *rb = red + (size_t)sl * RS;
+        if ((lane & ((1 << SH) - 1)) == 0) rb[cw * RV + (lane >> SH)] = tot;
+        if (cw == 0 && lane < NT) {
+          rb[CW * RV + lane] = pick<NT>(pscale, lane);
+          rb[CW * RV + 4 + lane] = __int_as_float(pick<NT>(pair_of, lane));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfull[sl]);
       }
     }
   }
-  pdl_launch_dependents();
-}
-
-// ------------------------------------------------------------------ down
-// Work unit = two consecutive output rows of one expert (H is even).
-template <int NT>
-__global__ void __launch_bounds__(kThreads) gemv_down_kernel(MoeArgs a) {
-  pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t warps_total = (int64_t)gridDim.x * kWarps;
-  const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int64_t I = a.I, H = a.H;
-  const int64_t per_expert = H / 2;
-  const int64_t units = (int64_t)(*a.n_active) * per_expert;
-  const int64_t u0 = units * gw / warps_total, u1 = units * (gw + 1) / warps_total;
-  const int nchunks = (int)(I / 32);
-
-  for (int64_t u = u0; u < u1; ++u) {
-    const int e = a.active[u / per_expert];
-    const int64_t n = (u % per_expert) * 2;
-    const int off = a.offsets[e], cnt = a.counts[e];
-    const uint8_t *p0 = a.w_dn + ((int64_t)e * H + n) * (I / 2);
-    const uint8_t *p1 = p0 + I / 2;
-    const uint8_t *s0r = a.s_dn + ((int64_t)e * H + n) * (I / 16);
-    const uint8_t *s1r = s0r + I / 16;
-    const float g = __ldg(a.g_dn + e);
-    for (int t0 = 0; t0 < cnt; t0 += NT) {
-      const int nt = min(NT, cnt - t0);
-      const __nv_bfloat16 *hr[NT];
-#pragma unroll
-      for (int i = 0; i < NT; ++i) hr[i] = a.h + (int64_t)(off + t0 + min(i, nt - 1)) * I;
-      float2 a0[NT], a1[NT];
-#pragma unroll
-      for (int i = 0; i < NT; ++i) a0[i] = a1[i] = make_float2(0.f, 0.f);
-#pragma unroll 2
-      for (int c = lane; c < nchunks; c += 32) {
-        const uint4 q0 = ldg_stream(p0 + 16 * c);
-        const uint4 q1 = ldg_stream(p1 + 16 * c);
-        float s00, s01, s10, s11;
-        scales2(s0r, c, s00, s01);
-        scales2(s1r, c, s10, s11);
-#pragma unroll
-        for (int i = 0; i < NT; ++i) {
-          if (i < nt) {
-            uint4 hv[4];
-            load_x_chunk(hr[i], c, hv);
-            a0[i] = chunk_dot(q0, s00, s01, hv, a0[i]);
-            a1[i] = chunk_dot(q1, s10, s11, hv, a1[i]);
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        if (i < nt) {
-          const float d0 = warp_sum(a0[i].x + a0[i].y);
-          const float d1 = warp_sum(a1[i].x + a1[i].y);
-          if (lane == 0) {
-            const int r = off + t0 + i;
-            const float wk = __ldg(a.w + a.perm[r]) * g;
-            *reinterpret_cast<float2 *>(a.y + (int64_t)r * H + n) = make_float2(wk * d0, wk * d1);
-          }
-        }
-      }
+  named_sync(2, nthreads_cf);   // every y of this CTA is in yk
+  // combine in ascending k: out[t, n] = sum_k y(slot(t, k))[n]
+  const int ctid = threadIdx.x - 32;
+  const int nbr = n1 - n0;
+  for (int o = ctid; o < T * nbr; o += nthreads_cf) {
+    const int t = o / nbr, rr = o % nbr;
+    float acc = 0.f;
+    for (int k = 0; k < K; ++k) {
+      const int sl = slot_of[t * K + k];
+      if (sl >= 0) acc += yk[(size_t)sl * nb + rr];
     }
+    a.out[(int64_t)t * H + n0 + rr] = __float2bfloat16_rn(acc);
   }
-  pdl_launch_dependents();
 }
 
-int gemv_grid() { return kNumSMs * 4; }
+int g_num_sms = 0;
+
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = kNumSMs;
+  }
+  return g_num_sms;
+}
+
+// Blocks of kernel k that fit on one SM at once with this block size and shared memory.
+template <typename Kern>
+int resident_blocks(Kern k, int threads, size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return -1;
+  }
+  int nb = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k, threads, smem);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return -1;
+  }
+  return nb;
+}
+
+int tokens_per_group(int64_t T) { return T <= 1 ? 1 : (T <= 16 ? 2 : 4); }
+
+template <int NT, int P, int S>
+int launch_gateup_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
+  const int CW = (int)ceil_div(a.H, 1024);
+  const uint32_t stage_bytes = (uint32_t)(2 * P * (a.H / 2) + 2 * span_bytes(P * (a.H / 16)));
+  const int n = (int)(a.T * a.K);
+  const Smem L = smem_layout(S, stage_bytes, CW, 2 * P * NT, n, (int)a.E, 0);
+  // the CTAs split the work evenly, so all of them must be resident at once
+  const int fit = resident_blocks(gemv_gateup_kernel<NT, P, S>, 32 * (CW + 2), L.total);
+  if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
+  return launch_pdl(gemv_gateup_kernel<NT, P, S>, dim3(num_sms() * min(ctas_per_sm, fit)),
+                    dim3(32 * (CW + 2)), L.total, s, a, stage_bytes);
+}
+
+template <int NT, int RD, int S>
+int launch_down_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
+  const int CW = (int)ceil_div(a.I, 512);
+  const uint32_t stage_bytes = (uint32_t)(RD * (a.I / 2) + span_bytes(RD * (a.I / 16)));
+  const int n = (int)(a.T * a.K);
+  // enough CTAs for the GPU, and few enough rows per CTA that the per-pair results fit
+  int64_t ctas = (int64_t)num_sms() * ctas_per_sm;
+  const int64_t max_nb = max64(1, (32 * 1024) / (4 * (n > 1 ? n : 1)));
+  ctas = max64(ctas, ceil_div(a.H, max_nb));
+  const int nb = (int)ceil_div(a.H, ctas);
+  ctas = ceil_div(a.H, nb);
+  const Smem L = smem_layout(S, stage_bytes, CW, RD * NT, n, (int)a.E, n * nb);
+  const int fit = resident_blocks(gemv_down_kernel<NT, RD, S>, 32 * (CW + 2), L.total);
+  if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
+  return launch_pdl(gemv_down_kernel<NT, RD, S>, dim3((unsigned)ctas), dim3(32 * (CW + 2)),
+                    L.total, s, a, stage_bytes, nb);
+}
 
 }  // namespace
 
+bool gemv_supported(int64_t T, int64_t H, int64_t I, int64_t K) {
+  return T * K <= kGemvMaxPairs && H <= 1024 * kMaxConsumerWarps && I <= 512 * kMaxConsumerWarps;
+}
+
 int launch_gemv_gateup(const MoeArgs &a, cudaStream_t s) {
-  const dim3 grid(gemv_grid()), block(kThreads);
-  if (a.T <= 1) return launch_pdl(gemv_gateup_kernel<1>, grid, block, 0, s, a);
-  if (a.T <= 16) return launch_pdl(gemv_gateup_kernel<2>, grid, block, 0, s, a);
-  return launch_pdl(gemv_gateup_kernel<4>, grid, block, 0, s, a);
+  switch (tokens_per_group(a.T)) {
+    case 1: return launch_gateup_cfg<1, kPairs, kStages>(a, s, NVFP4_GEMV_CTAS_PER_SM);
+    case 2: return launch_gateup_cfg<2, kPairs, kStages>(a, s, NVFP4_GEMV_CTAS_PER_SM);
+    default: return launch_gateup_cfg<4, kPairs, kStages>(a, s, 2);
+  }
 }
 
 int launch_gemv_down(const MoeArgs &a, cudaStream_t s) {
-  const dim3 grid(gemv_grid()), block(kThreads);
-  if (a.T <= 1) return launch_pdl(gemv_down_kernel<1>, grid, block, 0, s, a);
-  if (a.T <= 16) return launch_pdl(gemv_down_kernel<2>, grid, block, 0, s, a);
-  return launch_pdl(gemv_down_kernel<4>, grid, block, 0, s, a);
+  switch (tokens_per_group(a.T)) {
+    case 1: return launch_down_cfg<1, kDownRows, kStages>(a, s, NVFP4_GEMV_DOWN_CTAS_PER_SM);
+    case 2: return launch_down_cfg<2, kDownRows, kStages>(a, s, NVFP4_GEMV_DOWN_CTAS_PER_SM);
+    default: return launch_down_cfg<4, kDownRows, kStages>(a, s, 3);
+  }
 }
 
 }  // namespace nvfp4

@@ -40,9 +40,11 @@ struct WorkspaceLayout {
 WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
 constexpr int kGatherPadRows = 256;
 
-// GEMV path (decode.cu) and combine (combine.cu)
+// GEMV path (decode.cu): routing fused into both kernels, combine fused into the second
+bool gemv_supported(int64_t T, int64_t H, int64_t I, int64_t K);
 int launch_gemv_gateup(const MoeArgs &a, cudaStream_t s);
 int launch_gemv_down(const MoeArgs &a, cudaStream_t s);
+// combine of the GEMM path (combine.cu)
 int launch_combine(const MoeArgs &a, cudaStream_t s);
 // GEMM path (gemm.cu)
 int launch_gemm_gateup(const MoeArgs &a, cudaStream_t s);   // gather + gate/up + SwiGLU

@@ -111,7 +111,7 @@ NVFP4_API int nvfp4_cast_f32(const float *in, int64_t n, uint8_t *e4m3, uint8_t 
  *   w_dn     [E, H, I/2] u8         s_dn [E, H, I/16] E4M3     g_dn [E] fp32
  *   out      [T, H] bf16
  * Limits: H % 64 == 0, I % 64 == 0, 1 <= K <= 16, E <= 1024, T*K < 2^31.
- * Alignment: x, w_gu, w_dn, out and workspace 16 bytes; s_gu, s_dn 2 bytes (EINVAL /
+ * Alignment: x, w_gu, s_gu, w_dn, s_dn, out and workspace 16 bytes (EINVAL /
  * EWORKSPACE otherwise).
  * The call picks a memory-bound GEMV path for small T and a tensor-core grouped GEMM path
  * otherwise; both compute the same function.  It never synchronises with the host and
@@ -144,7 +144,8 @@ NVFP4_API int moe_nvfp4_forward_path(const __nv_bfloat16 *x, const int32_t *topk
  * cudaEvent_t (created by the caller, timing enabled) that are recorded on `stream`:
  * [0] before the route step, [1] after it, [2] after the gate/up + SwiGLU step, [3] after
  * the down step, [4] after the combine.  The events sit between the kernels, so the
- * kernels do not overlap their neighbours as they do in an unmarked call.
+ * kernels do not overlap their neighbours as they do in an unmarked call.  Under stream
+ * capture the marks are recorded as external events, so they time each graph replay.
  * Errors as moe_nvfp4_forward_path, plus EINVAL for a null event. */
 NVFP4_API int moe_nvfp4_forward_profiled(const __nv_bfloat16 *x, const int32_t *topk_ids,
                                          const float *topk_w, int64_t T, int64_t H, int64_t I,
