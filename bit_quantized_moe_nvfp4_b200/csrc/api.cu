@@ -49,7 +49,7 @@ WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int
   L.tile_prefix = take(4 * (size_t)(E + 1));
   L.perm = take(4 * TK);
   L.inv = take(4 * TK);
-  L.h = take(2 * TK * (size_t)I);
+  L.h = take(2 * (TK + kGatherPadRows) * (size_t)I);   // rows past T*K: tile overhang
   L.y = take(4 * TK * (size_t)H);
   L.xs = take(2 * (TK + kGatherPadRows) * (size_t)H);
   L.total = o;
