@@ -52,6 +52,7 @@ WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int
   L.h = take(2 * (TK + kGatherPadRows) * (size_t)I);   // rows past T*K: tile overhang
   L.y = take(4 * TK * (size_t)H);
   L.xs = take(2 * (TK + kGatherPadRows) * (size_t)H);
+  L.xscale = take(4 * TK);
   L.total = o;
   return L;
 }
@@ -147,7 +148,8 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   a.inv = reinterpret_cast<int32_t *>(ws + L.inv);
   a.h = reinterpret_cast<__nv_bfloat16 *>(ws + L.h);
   a.y = reinterpret_cast<float *>(ws + L.y);
-  a.xs = reinterpret_cast<__nv_bfloat16 *>(ws + L.xs);
+  a.xs = reinterpret_cast<__half *>(ws + L.xs);
+  a.xscale = reinterpret_cast<float *>(ws + L.xscale);
 
   if (path == NVFP4_PATH_AUTO)
     path = (T <= kGemvMaxTokens && gemv_supported(T, H, I, K)) ? NVFP4_PATH_GEMV

@@ -117,4 +117,18 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// ------------------------------------------------------------------ f16 activation scaling
+// Activations enter f16 tensor/FMA operands after scaling by 2^p with p = 14 - floor(log2 m),
+// m the row's largest magnitude, so m * 2^p lies in [2^14, 2^15).  bf16 has 8 significant
+// bits and f16 11, so the rounding to f16 is exact for every element above 2^-31 * m.
+__device__ __forceinline__ float exp2i(int p) { return __uint_as_float((uint32_t)(p + 127) << 23); }
+
+__device__ __forceinline__ int prescale_exponent(float m) {
+  if (!(m > 0.0f)) return 0;
+  const int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 127;  // floor(log2 m) for normals
+  int p = 14 - e;
+  p = max(-100, min(100, p));
+  return p;
+}
+
 }  // namespace nvfp4

@@ -103,17 +103,6 @@ __device__ __forceinline__ V pick(const V (&v)[N], int i) {
   return r;
 }
 
-// Power of two 2^p as fp32, p in [-126, 127].
-__device__ __forceinline__ float exp2i(int p) { return __uint_as_float((uint32_t)(p + 127) << 23); }
-
-// Scale exponent for a token whose largest magnitude is m: m * 2^p lands in [2^14, 2^15).
-__device__ __forceinline__ int prescale_exponent(float m) {
-  if (!(m > 0.0f)) return 0;
-  const int e = (int)((__float_as_uint(m) >> 23) & 0xFF) - 127;  // floor(log2 m) for normals
-  int p = 14 - e;
-  p = max(-100, min(100, p));
-  return p;
-}
 
 // 2 x f32 -> f16x2 (round to nearest even)
 __device__ __forceinline__ uint32_t f16x2_rn(float lo, float hi) {

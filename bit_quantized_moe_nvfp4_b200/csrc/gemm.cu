@@ -4,24 +4,28 @@
 // per 16 elements), 256 experts, 8 active per token.  With many tokens per expert each
 // projection is a dense contraction per expert, run on the tensor cores:
 //
-//   gather:  xs[r] = x[token of routed pair r]           (pairs in expert order)
-//   gate/up: D = W_gu[e] (rows j0..j0+63 gate, same rows up) . xs[slots of e]^T
-//            h[slot, j] = bf16( silu(g_gu*D_gate) * g_gu*D_up )
-//   down:    D = W_dn[e] (128 rows) . h[slots of e]^T
+//   gather:  xs[r] = f16(x[token of pair r] * 2^p_r)   (pairs in expert order, exact
+//            per-row power-of-two scale, xscale[r] = 2^-p_r)
+//   gate/up: D = W_gu[e] (rows j0..j0+63 gate, same rows up) . xs[slots of e]^T   (f16 MMA)
+//            h[slot, j] = bf16( silu(g_gu*xscale*D_gate) * g_gu*xscale*D_up )
+//   down:    D = W_dn[e] (128 rows) . h[slots of e]^T                          (bf16 MMA)
 //            y[slot, n] = w[pair] * g_dn * D
 //   combine (combine.cu): out[t] = bf16( sum over k of y[slot(t, k)] )
 //
-// One persistent CTA per SM walks the tiles (expert, 256-slot n-tile, 128-row m-tile) with
+// One persistent CTA per SM walks the tiles (expert, 224-slot n-tile, 128-row m-tile) with
 // warp-specialised roles:
 //   warp 0     TMA producer: packed weight rows (2 boxes of 64 rows x 32 bytes) and the
-//              activation tile (256 rows x 64 bf16, 128-byte swizzle) per 64-wide K step;
-//   warp 1     allocates TMEM and issues tcgen05.mma (M=128, N<=256, K=16, fp32 in TMEM);
-//   warps 2-5  dequantize: one weight row per thread, E2M1 x E4M3 -> bf16 (exact: at most 6
-//              significant bits) written into the K-major SW128 operand tile;
-//   warps 6-9  epilogue: tcgen05.ld of the accumulator, global scale, SwiGLU or routing
+//              activation tile (224 rows x 64 elements, 128-byte swizzle) per 64-wide K step;
+//   warp 1     allocates TMEM and issues tcgen05.mma (M=128, N<=224, K=16, fp32 in TMEM)
+//              with the weight operand read from TMEM and the activations from shared memory;
+//   warps 2-9  dequantize: half a weight row per thread, E2M1 x E4M3 -> f16 (gate/up) or
+//              bf16 (down), exact either way (at most 6 significant bits), stored straight
+//              into the thread's TMEM lane (tcgen05.st), so the dequantized operand never
+//              touches shared memory;
+//   warps 10-13 epilogue: tcgen05.ld of the accumulator, global scale, SwiGLU or routing
 //              weight, stores.
-// Accumulators are double-buffered in TMEM (2 x 256 columns), so the epilogue of one tile
-// overlaps the main loop of the next.  The weights sit on M ("swap AB") because experts get
+// Accumulators are double-buffered in TMEM (2 x 224 columns, next to two 32-column weight
+// operand slots), so the epilogue of one tile overlaps the main loop of the next.  The weights sit on M ("swap AB") because experts get
 // anywhere from 0 to thousands of tokens: the token count only changes N.
 #include <cuda.h>
 
@@ -32,23 +36,45 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int BM = 128;          // weight rows per tile
-constexpr int BN = 256;          // token slots per tile (largest N of one MMA)
-constexpr int BK = 64;           // reduction elements per stage (128-byte bf16 rows)
-constexpr int kS = 4;            // stages of packed weights + activation tiles
-constexpr int kSA = 2;           // dequantized weight tiles
-constexpr int kThreads = 320;    // 10 warps
-constexpr uint32_t kTmemCols = 512;
+// Pipeline depth and dequant width (compile-time tunables; defaults measured on B200).
+#ifndef NVFP4_GEMM_STAGES
+#define NVFP4_GEMM_STAGES 6
+#endif
+#ifndef NVFP4_GEMM_BN
+#define NVFP4_GEMM_BN 224
+#endif
+#ifndef NVFP4_GEMM_A_SLOTS
+#define NVFP4_GEMM_A_SLOTS 2
+#endif
+#ifndef NVFP4_GEMM_DEQUANT_WARPS
+#define NVFP4_GEMM_DEQUANT_WARPS 8
+#endif
+constexpr int BM = 128;          // weight rows per tile (TMEM lanes)
+constexpr int BN = NVFP4_GEMM_BN;   // token slots per tile (MMA N, multiple of 16)
+constexpr int BK = 64;           // reduction elements per stage
+constexpr int kS = NVFP4_GEMM_STAGES;           // stages: packed weights + activation tile
+constexpr int kSA = NVFP4_GEMM_A_SLOTS;         // weight operand slots in TMEM
+constexpr int kDQW = NVFP4_GEMM_DEQUANT_WARPS;  // 4 (full rows) or 8 (half rows)
+constexpr int kWarpEpi = 2 + kDQW;              // first of the 4 epilogue warps
+constexpr int kThreads = 32 * (kWarpEpi + 4);
+static_assert(kDQW == 4 || kDQW == 8, "dequant warps: 4 or 8");
 
-constexpr uint32_t kBBytes = BN * BK * 2;     // 32 KB
-constexpr uint32_t kABytes = BM * BK * 2;     // 16 KB
-constexpr uint32_t kPBytes = BM * BK / 2;     // 4 KB packed
+// Tensor memory: two fp32 accumulators of BN columns, then kSA weight operands of BK/2
+// columns (64 16-bit values of a row per lane) -- 2*224 + 2*32 = 512 columns.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemA = 2 * BN;
+constexpr uint32_t kACols = BK / 2;
+static_assert(kTmemA + kSA * kACols <= kTmemCols, "TMEM budget");
+
+constexpr uint32_t kBBytes = BN * BK * 2;     // activation tile (128-byte swizzle)
+static_assert(kBBytes % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
+constexpr uint32_t kPBytes = BM * BK / 2;     // 4 KB packed weights
 constexpr uint32_t kSmemB = 0;
-constexpr uint32_t kSmemA = kSmemB + kS * kBBytes;
-constexpr uint32_t kSmemP = kSmemA + kSA * kABytes;
+constexpr uint32_t kSmemP = kSmemB + kS * kBBytes;
 constexpr uint32_t kSmemBars = kSmemP + kS * kPBytes;
 constexpr uint32_t kSmemMisc = kSmemBars + 8 * (2 * kS + 2 * kSA + 4);
 constexpr uint32_t kSmemTotal = kSmemMisc + 16 + 1024;   // + alignment slack
+static_assert(kSmemTotal <= 227 * 1024, "shared memory budget");
 
 struct GemmParams {
   MoeArgs a;
@@ -89,29 +115,50 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, int tile, int
 
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
 
-// ------------------------------------------------------------------ dequantize one row
-// 64 E2M1 codes (32 bytes) with 4 E4M3 block scales -> 64 bf16 in the K-major SW128 tile.
-__device__ __forceinline__ void dequant_row(const uint4 (&q)[2], uint32_t scales4, unsigned char *a_tile,
-                                            int arow) {
-  const uint32_t words[8] = {q[0].x, q[0].y, q[0].z, q[0].w, q[1].x, q[1].y, q[1].z, q[1].w};
-  const uint32_t s01 = e4m3x2_to_f16x2(scales4 & 0xFFFFu);
-  const uint32_t s23 = e4m3x2_to_f16x2(scales4 >> 16);
-  unsigned char *row = a_tile + (arow >> 3) * 1024 + (arow & 7) * 128;
+// ------------------------------------------------------------------ dequantize
+// NW packed words (8 E2M1 codes each) with their NW/2 block scales (one byte per 16
+// elements, low bytes first) -> 4*NW packed 16-bit pairs, each the exact product e2m1*e4m3:
+//   f16:  the hardware E2M1 -> f16 convert, then one f16 multiply by the scale.
+//   bf16: the f16 magnitude bits shifted right by 3 read as bf16 are |q| * 2^-112 (the exponent
+//         field widens from 5 to 8 bits; q has one mantissa bit, so nothing is lost), one
+//         bf16 multiply by s * 2^112 (exact, below 2^121) gives |q| * s, and the sign bit is
+//         copied back.  This keeps the conversion on the integer pipes.
+template <bool F16, int NW>
+__device__ __forceinline__ void dequant_words(const uint32_t (&words)[NW], uint32_t scales,
+                                              uint32_t (&out)[4 * NW]) {
+  uint32_t sb[NW / 2];   // per block: the scale in both halves, f16 or bf16(s * 2^112)
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {          // 16-byte output chunk c = elements 8c..8c+7
-    const uint32_t sb = (c < 4) ? ((c < 2) ? __byte_perm(s01, 0, 0x1010) : __byte_perm(s01, 0, 0x3232))
-                                : ((c < 6) ? __byte_perm(s23, 0, 0x1010) : __byte_perm(s23, 0, 0x3232));
+  for (int b = 0; b < NW / 2; b += 2) {
+    const uint32_t s2 = e4m3x2_to_f16x2((scales >> (8 * b)) & 0xFFFFu);
+    const uint32_t sh[2] = {__byte_perm(s2, 0, 0x1010), __byte_perm(s2, 0, 0x3232)};
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (b + k >= NW / 2) break;
+      if (F16) {
+        sb[b + k] = sh[k];
+      } else {
+        const float sv = f16_lo(sh[k]) * 5.192296858534828e33f;   // s * 2^112
+        sb[b + k] = pack_bf16x2(sv, sv);
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < NW; ++c) {
     uint32_t h[4];
     e2m1x8_to_f16x2x4(words[c], h);
-    uint32_t o[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      // q * s is exact in f16 and in bf16 (at most 6 significant bits, within range)
-      __half2 v = __hmul2(*reinterpret_cast<__half2 *>(&h[p]), *reinterpret_cast<const __half2 *>(&sb));
-      const float2 f = __half22float2(v);
-      o[p] = pack_bf16x2(f.x, f.y);
+      const uint32_t s2 = sb[c >> 1];
+      if (F16) {
+        __half2 v = __hmul2(*reinterpret_cast<__half2 *>(&h[p]), *reinterpret_cast<const __half2 *>(&s2));
+        out[4 * c + p] = *reinterpret_cast<uint32_t *>(&v);
+      } else {
+        uint32_t mag = (h[p] >> 3) & 0x0FFF0FFFu;
+        __nv_bfloat162 v = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&mag),
+                                   *reinterpret_cast<const __nv_bfloat162 *>(&s2));
+        out[4 * c + p] = *reinterpret_cast<uint32_t *>(&v) | (h[p] & 0x80008000u);
+      }
     }
-    *reinterpret_cast<uint4 *>(row + ((c ^ (arow & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -122,11 +169,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem =
       smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);   // 1024-byte aligned
+  // Stage s holds packed weights P[s] and the activation tile B[s]; the weight operand of
+  // K step kg lives in TMEM slot kg % kSA.
+  //   full[s]    TMA bytes of P[s] and B[s] have landed            (producer -> dequant)
+  //   freeb[s]   the MMAs reading B[s] are done                    (MMA commit -> producer)
+  //   afull[sa]  TMEM weight slot sa is written (P, B landed)      (dequant -> MMA)
+  //   afree[sa]  the MMAs reading TMEM slot sa are done            (MMA commit -> dequant)
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kSmemBars);
-  uint64_t *empty = full + kS;
-  uint64_t *afull = empty + kS;
-  uint64_t *aempty = afull + kSA;
-  uint64_t *accfull = aempty + kSA;      // [2]
+  uint64_t *freeb = full + kS;
+  uint64_t *afull = freeb + kS;
+  uint64_t *afree = afull + kSA;
+  uint64_t *accfull = afree + kSA;       // [2]
   uint64_t *accempty = accfull + 2;      // [2]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmemMisc);
   int *abort = reinterpret_cast<int *>(smem + kSmemMisc + 4);
@@ -138,11 +191,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort = 0;
     for (int s = 0; s < kS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&freeb[s], 1);
     }
     for (int s = 0; s < kSA; ++s) {
-      mbar_init(&afull[s], 4);
-      mbar_init(&aempty[s], 1);
+      mbar_init(&afull[s], kDQW);
+      mbar_init(&afree[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&accfull[s], 1);
@@ -162,7 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kblocks = p.K / BK;
   const int64_t I = a.I, H = a.H;
 
+  // Bounded wait; after any wait of the CTA has given up, later slow waits return at once.
   auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
     if (*(volatile int *)abort) return false;
     if (mbar_wait(bar, parity)) return true;
     *(volatile int *)abort = 1;
@@ -186,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int kb = 0; kb < kblocks; ++kb, ++kg) {
           const int s = kg % kS;
-          if (kg >= kS && !wait(&empty[s], ((kg / kS) - 1) & 1)) break;
+          if (kg >= kS && !wait(&freeb[s], ((kg / kS) - 1) & 1)) break;
           if (*(volatile int *)abort) break;
           mbar_arrive_expect_tx(&full[s], kPBytes + kBBytes);
           unsigned char *pk = smem + kSmemP + s * kPBytes;
@@ -209,67 +264,110 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tc >= 2 && !wait(&accempty[acc], ((tc >> 1) - 1) & 1)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        const uint32_t idesc = idesc_bf16_f32(BM, max(16, round16(t.nvalid)));
+        const int nmma = max(16, round16(t.nvalid));
+        const uint32_t idesc = p.mode == 0 ? idesc_f16_f32(BM, nmma) : idesc_bf16_f32(BM, nmma);
         for (int kb = 0; kb < kblocks; ++kb, ++kg) {
           const int s = kg % kS, sa = kg % kSA;
-          const bool ok = wait(&full[s], (kg / kS) & 1) && wait(&afull[sa], (kg / kSA) & 1);
+          const bool ok = wait(&afull[sa], (kg / kSA) & 1);   // implies full[s]
           tc_fence_after();
           if (ok) {
-            const uint32_t a_addr = smem_u32(smem + kSmemA + sa * kABytes);
-            const uint32_t b_addr = smem_u32(smem + kSmemB + s * kBBytes);
+            const uint32_t a_tmem = tmem_base + kTmemA + sa * kACols;
+            const uint64_t db = smem_desc_sw128(smem_u32(smem + kSmemB + s * kBBytes));
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_bf16(d_tmem, smem_desc_sw128(a_addr + 32 * kk), smem_desc_sw128(b_addr + 32 * kk),
-                        idesc, kb > 0 || kk > 0);
+            for (int kk = 0; kk < BK / 16; ++kk)   // K=16: 8 TMEM columns, 32 bytes of B
+              umma_ts(d_tmem, a_tmem + 8 * kk, db + 2 * kk, idesc, kb > 0 || kk > 0);
           }
-          umma_commit(&empty[s]);
-          umma_commit(&aempty[sa]);
+          umma_commit(&freeb[s]);
+          umma_commit(&afree[sa]);
         }
         umma_commit(&accfull[acc]);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < kWarpEpi) {
     // ---------------------------------------------------------------- dequantize
-    const int dt = threadIdx.x - 64;            // packed row of the tile handled here
+    // Warp w writes TMEM lanes 32*(w%4)..+31: lane L holds weight-operand row L.  With 8
+    // warps, the second four write the upper half of each row's 64 elements.
+    constexpr int kPerRow = kDQW / 4;            // threads per row (1 or 2)
+    constexpr int NW = 8 / kPerRow;              // packed words per thread per step
+    const int q = warp & 3;
+    const int part = (warp - 2) / 4;             // 0, or 1 for the second four warps
+    const int L = q * 32 + lane;                 // operand row = TMEM lane
     int kg = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const TileInfo t = tile_info(p, tile, n_act);
       int64_t wrow;
-      int arow;
+      int prow;            // row of the packed tile feeding operand row L
       bool valid = true;
       if (p.mode == 0) {
-        const int jj = dt & 63;
-        wrow = (int64_t)t.e * 2 * I + (dt < 64 ? 0 : I) + t.mt * 64 + jj;
-        arow = 2 * jj + (dt < 64 ? 0 : 1);       // gate j at row 2j, up j at row 2j+1
+        const int jj = L >> 1;                   // gate j at row 2j, up j at row 2j+1
+        prow = (L & 1) ? 64 + jj : jj;
+        wrow = (int64_t)t.e * 2 * I + ((L & 1) ? I : 0) + t.mt * 64 + jj;
       } else {
-        const int64_t n = (int64_t)t.mt * BM + dt;
+        const int64_t n = (int64_t)t.mt * BM + L;
         valid = n < H;
+        prow = L;
         wrow = (int64_t)t.e * H + n;
-        arow = dt;
       }
+      // Block scales of this row: 4 bytes per K step, fetched 16 bytes (four steps) at a
+      // time, two groups ahead.  Rows whose scale run is not 16-byte aligned take 4-byte loads.
       const uint8_t *srow = p.scales + wrow * (p.K / 16);
-      uint32_t sc_next = valid ? __ldg(reinterpret_cast<const uint32_t *>(srow)) : 0u;
+      const bool wide = (p.K % 256) == 0;
+      auto group = [&](int g) -> uint4 {
+        if (!valid || 4 * g >= kblocks) return make_uint4(0, 0, 0, 0);
+        if (wide) return __ldg(reinterpret_cast<const uint4 *>(srow) + g);
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(srow) + 4 * g;
+        const int left = kblocks - 4 * g;
+        return make_uint4(__ldg(w), left > 1 ? __ldg(w + 1) : 0u, left > 2 ? __ldg(w + 2) : 0u,
+                          left > 3 ? __ldg(w + 3) : 0u);
+      };
+      uint4 g0 = group(0), g1 = group(1), g2 = group(2);
       for (int kb = 0; kb < kblocks; ++kb, ++kg) {
         const int s = kg % kS, sa = kg % kSA;
-        const uint32_t sc = sc_next;
-        if (kb + 1 < kblocks && valid)
-          sc_next = __ldg(reinterpret_cast<const uint32_t *>(srow) + kb + 1);
-        bool ok = wait(&full[s], (kg / kS) & 1);
-        if (kg >= kSA) ok = wait(&aempty[sa], ((kg / kSA) - 1) & 1) && ok;
-        if (ok) {
-          const uint4 *src = reinterpret_cast<const uint4 *>(smem + kSmemP + s * kPBytes + dt * (BK / 2));
-          uint4 q[2] = {src[0], src[1]};
-          if (!valid) q[0] = q[1] = make_uint4(0, 0, 0, 0);
-          dequant_row(q, sc, smem + kSmemA + sa * kABytes, arow);
+        if (kb > 0 && (kb & 3) == 0) {
+          g0 = g1;
+          g1 = g2;
+          g2 = group((kb >> 2) + 2);
         }
-        fence_proxy_async_smem();
+        const int w4 = kb & 3;
+        const uint32_t sc = w4 == 0 ? g0.x : (w4 == 1 ? g0.y : (w4 == 2 ? g0.z : g0.w));
+        bool ok = wait(&full[s], (kg / kS) & 1);
+        if (kg >= kSA) ok = wait(&afree[sa], ((kg / kSA) - 1) & 1) && ok;
+        tc_fence_after();
+        uint32_t w[NW];
+        const uint32_t *src32 =
+            reinterpret_cast<const uint32_t *>(smem + kSmemP + s * kPBytes + prow * (BK / 2)) + part * NW;
+#pragma unroll
+        for (int i = 0; i < NW; i += 4) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(src32 + i);
+          w[i] = v.x;
+          w[i + 1] = v.y;
+          w[i + 2] = v.z;
+          w[i + 3] = v.w;
+        }
+        if (!valid || !ok)
+#pragma unroll
+          for (int i = 0; i < NW; ++i) w[i] = 0u;
+        const uint32_t scp = sc >> (8 * (NW / 2) * part);    // this part's block scales
+        uint32_t o[4 * NW];
+        if (p.mode == 0)
+          dequant_words<true, NW>(w, scp, o);
+        else
+          dequant_words<false, NW>(w, scp, o);
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + kTmemA + sa * kACols +
+                               part * (kACols / kPerRow);
+        if (NW == 8)
+          tmem_st32(taddr, *reinterpret_cast<uint32_t(*)[32]>(o));
+        else
+          tmem_st16(taddr, *reinterpret_cast<uint32_t(*)[16]>(o));
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&afull[sa]);
       }
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;                     // TMEM lane quarter of this warp
+    const int q = warp & 3;                     // TMEM lane quarter of this warp (the four
+                                                // epilogue warps are consecutive)
     const int m = q * 32 + lane;                // accumulator row (TMEM lane)
     int tc = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
@@ -284,9 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c0, v);
         if (p.mode == 0) {
           const int64_t j = (int64_t)t.mt * 64 + (m >> 1);
+          const float xl = (c0 + lane < t.nvalid) ? a.xscale[t.slot0 + c0 + lane] * g : 0.f;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float val = __uint_as_float(v[c]) * g;
+            const float val = __uint_as_float(v[c]) * __shfl_sync(0xFFFFFFFFu, xl, c);
             const float other = __shfl_xor_sync(0xFFFFFFFFu, val, 1);
             if (!(lane & 1) && c0 + c < t.nvalid) {
               const float hv = silu_f32(val) * other;       // val = gate, other = up
@@ -322,18 +421,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ gather
-// xs[r] = x[perm[r] / K] for the routed pairs (one warp per row, 16-byte copies).
+// xs[r] = f16(x[perm[r] / K] * 2^p_r), xscale[r] = 2^-p_r, for the routed pairs: one warp
+// per row, 16-byte accesses; the row is read twice (largest magnitude, then convert), the
+// second time from cache.
 __global__ void __launch_bounds__(256) gather_kernel(MoeArgs a) {
   pdl_wait();
   const int64_t H = a.H, K = a.K;
   const int n_valid = a.offsets[a.E];
   const int vec = (int)(H / 8);
+  const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * 8;
   for (int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); r < n_valid; r += warps) {
     const int64_t t = a.perm[r] / K;
     const uint4 *src = reinterpret_cast<const uint4 *>(a.x + t * H);
     uint4 *dst = reinterpret_cast<uint4 *>(a.xs + r * H);
-    for (int i = threadIdx.x & 31; i < vec; i += 32) dst[i] = __ldg(src + i);
+    float m = 0.f;
+    for (int i = lane; i < vec; i += 32) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[k])), fabsf(bf16_hi(w[k]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const int p = prescale_exponent(m);
+    const float sc = exp2i(p);
+    for (int i = lane; i < vec; i += 32) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __half2 hv = __floats2half2_rn(bf16_lo(w[k]) * sc, bf16_hi(w[k]) * sc);
+        o[k] = *reinterpret_cast<uint32_t *>(&hv);
+      }
+      dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (lane == 0) a.xscale[r] = exp2i(-p);
   }
   pdl_launch_dependents();
 }
@@ -388,10 +512,11 @@ int launch_gemm(const MoeArgs &a, int mode, cudaStream_t s) {
                (uint64_t)(p.K / 2), (uint64_t)(a.E * rows_per_expert), BK / 2, 64,
                CU_TENSOR_MAP_SWIZZLE_NONE))
     return NVFP4_ECUDA;
-  // activations: [T*K + pad, K] bf16, boxes of BN rows x 64 elements, 128-byte swizzle
+  // activations: [T*K + pad, K] f16 (gate/up) or bf16 (down), boxes of BN rows x 64
+  // elements, 128-byte swizzle
   const uint64_t brows = (uint64_t)(a.T * a.K + kGatherPadRows);
-  if (make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, mode == 0 ? (const void *)a.xs
-                                                                     : (const void *)a.h,
+  if (make_map(&tb, mode == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+               2, mode == 0 ? (const void *)a.xs : (const void *)a.h,
                (uint64_t)p.K, brows, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return NVFP4_ECUDA;
   cudaError_t e =

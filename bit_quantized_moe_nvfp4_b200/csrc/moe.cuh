@@ -30,12 +30,14 @@ struct MoeArgs {
   int32_t *inv;               // [T*K]  position of pair t*K+k in perm
   __nv_bfloat16 *h;           // [T*K, I]   SwiGLU output, rows in perm order
   float *y;                   // [T*K, H]   w * g_dn * (W_dn h), rows in perm order
-  __nv_bfloat16 *xs;          // [T*K + pad, H]  x gathered in perm order (GEMM path)
+  __half *xs;                 // [T*K + pad, H]  x gathered in perm order, f16, row r
+                              //   scaled by 1/xscale[r] (GEMM path)
+  float *xscale;              // [T*K]  2^-p of each gathered row (GEMM path)
 };
 
 // Workspace carve-up (byte offsets, each 256-aligned).
 struct WorkspaceLayout {
-  size_t flag, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, total;
+  size_t flag, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, xscale, total;
 };
 WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
 constexpr int kGatherPadRows = 256;
