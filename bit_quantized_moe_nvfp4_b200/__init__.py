@@ -22,6 +22,7 @@ __all__ = [
     "nvfp4_quantize", "nvfp4_quantize_workspace_size", "nvfp4_dequantize", "nvfp4_cast_f32",
     "moe_nvfp4_route", "moe_nvfp4_workspace_size", "moe_nvfp4_forward",
     "moe_nvfp4_read_error_flag", "moe_nvfp4_forward_profiled", "alloc_moe_workspace",
+    "moe_nvfp4_forward_static",
 ]
 
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
@@ -56,6 +57,8 @@ def _load() -> ctypes.CDLL:
                                              P, P, P, P, P, P, P, P, SZ, I32, P, P]),
         "moe_nvfp4_read_error_flag": (I32, [P, P, P]),
         "moe_nvfp4_route": (I32, [P, I64, I64, I64, P, P, P, P, P, P]),
+        "moe_nvfp4_forward_static": (I32, [P, P, P, I64, I64, I64, I64, I64,
+                                           P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -227,6 +230,32 @@ def moe_nvfp4_forward_profiled(x, topk_ids, topk_w, w_gu, s_gu, g_gu, w_dn, s_dn
         _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, twoI // 2, E, K, _ptr(w_gu), _ptr(s_gu),
         _ptr(g_gu), _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(out), _ptr(workspace),
         workspace.numel(), int(path), arr, _stream(x.device)))
+    return out
+
+
+def moe_nvfp4_forward_static(x, topk_ids, topk_w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
+                             out=None, error_flag=None) -> torch.Tensor:
+    """The small-batch forward with the library's fixed scratch instead of a workspace
+    (see include/nvfp4_moe.h).  error_flag: optional int32 [1] device tensor that
+    receives the error bits.  Returns out bf16 [T,H]."""
+    _need(x, torch.bfloat16, "x")
+    _need(topk_ids, torch.int32, "topk_ids")
+    _need(topk_w, torch.float32, "topk_w")
+    for t, n in ((w_gu, "w_gu"), (s_gu, "s_gu"), (w_dn, "w_dn"), (s_dn, "s_dn")):
+        _need(t, torch.uint8, n)
+    _need(g_gu, torch.float32, "g_gu")
+    _need(g_dn, torch.float32, "g_dn")
+    if error_flag is not None:
+        _need(error_flag, torch.int32, "error_flag")
+    T, H = x.shape
+    K = topk_ids.shape[1]
+    E, twoI, _ = w_gu.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(_lib().moe_nvfp4_forward_static(
+        _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, twoI // 2, E, K, _ptr(w_gu), _ptr(s_gu),
+        _ptr(g_gu), _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(out),
+        _ptr(error_flag) if error_flag is not None else None, _stream(x.device)))
     return out
 
 

@@ -1,0 +1,106 @@
+// noalloc.cu -- moe_nvfp4_forward_static: the small-batch (GEMV) forward with a fixed,
+// library-owned scratch instead of a caller workspace.
+//
+// The pages define the MoE layer, not its memory management: this entry point has no
+// counterpart there.  It exists for callers that cannot hand the library any device memory
+// -- e.g. a decode loop that has committed every free byte of HBM to its KV-cache pool and
+// holds only the layer's own tensors, so it can neither allocate a workspace nor carve one
+// out of a buffer it owns.  The kernels are the ones moe_nvfp4_forward runs on its GEMV
+// path; only the scratch they write differs:
+//   h   [T*K, I] bf16   SwiGLU outputs, one row per routed pair    -> g_static_h below
+//   flag                error bits                                 -> the caller's pointer
+// Nothing in the scratch has to start at zero: the gate/up kernel writes every h row the
+// down kernel reads, and the flag is overwritten by each call.  The array keeps the rows of
+// the last call after it ends.  There is ONE array per device, shared by every call on that
+// device: calls on one stream are ordered and safe; calls that can overlap (different
+// streams or host threads on the same device) race on it.
+#include <mutex>
+
+#include "moe.cuh"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int64_t kStaticHElems = NVFP4_STATIC_MAX_H_ELEMS;   // 2^18 bf16 = 512 KB
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) __nv_bfloat16 g_static_h[kStaticHElems];
+
+std::mutex g_lookup_mu;
+void *g_static_h_addr[kMaxDevices] = {};
+
+// Device address of g_static_h on the current device, looked up once per device.  The
+// lookup may load this library's device code, which is why the first call on a device
+// has to come before any stream capture on it begins.
+int static_scratch(__nv_bfloat16 **h) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return NVFP4_ECUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return NVFP4_EINVAL;
+  std::lock_guard<std::mutex> lock(g_lookup_mu);
+  if (!g_static_h_addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_h);
+    if (e != cudaSuccess || !p) {
+      set_last_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      return NVFP4_ECUDA;
+    }
+    g_static_h_addr[dev] = p;
+  }
+  *h = static_cast<__nv_bfloat16 *>(g_static_h_addr[dev]);
+  return NVFP4_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *topk_ids,
+                                        const float *topk_w, int64_t T, int64_t H, int64_t I,
+                                        int64_t E, int64_t K, const uint8_t *w_gu,
+                                        const uint8_t *s_gu, const float *g_gu,
+                                        const uint8_t *w_dn, const uint8_t *s_dn,
+                                        const float *g_dn, __nv_bfloat16 *out,
+                                        int32_t *error_flag, cudaStream_t stream) {
+  if (!x || !topk_ids || !topk_w || !w_gu || !s_gu || !g_gu || !w_dn || !s_dn || !g_dn || !out)
+    return NVFP4_EINVAL;
+  if (T <= 0 || H <= 0 || I <= 0 || E <= 0 || K <= 0) return NVFP4_EINVAL;
+  if (H % 64 || I % 64 || K > 16 || E > kMaxExperts || T * K >= (int64_t(1) << 31))
+    return NVFP4_ESHAPE;
+  if (!aligned16(x) || !aligned16(w_gu) || !aligned16(w_dn) || !aligned16(out) ||
+      !aligned16(s_gu) || !aligned16(s_dn) ||
+      (reinterpret_cast<uintptr_t>(error_flag) & 3))
+    return NVFP4_EINVAL;
+  // the fixed scratch bounds the batch: T*K*I bf16 values of h
+  if (T * K > kStaticHElems / I || !gemv_supported(T, H, I, K)) return NVFP4_ESHAPE;
+
+  __nv_bfloat16 *h = nullptr;
+  if (int s = static_scratch(&h)) return s;
+
+  MoeArgs a = {};
+  a.x = x;
+  a.ids = topk_ids;
+  a.w = topk_w;
+  a.w_gu = w_gu;
+  a.s_gu = s_gu;
+  a.g_gu = g_gu;
+  a.w_dn = w_dn;
+  a.s_dn = s_dn;
+  a.g_dn = g_dn;
+  a.out = out;
+  a.T = T;
+  a.H = H;
+  a.I = I;
+  a.E = E;
+  a.K = K;
+  a.flag = error_flag;   // may be NULL: the kernels then skip the flag writes
+  a.h = h;
+  if (int s = launch_gemv_gateup(a, stream)) return s;
+  return launch_gemv_down(a, stream);
+}

@@ -12,16 +12,18 @@
  *
  * Conventions for every call:
  *   - Pointers are DEVICE pointers owned by the caller unless a parameter says "host".
- *     The library never allocates, frees or keeps memory; scratch comes from a caller
- *     workspace sized by the matching *_workspace_size() query.
+ *     The library never allocates or frees memory; scratch comes from a caller workspace
+ *     sized by the matching *_workspace_size() query, except for moe_nvfp4_forward_static,
+ *     which uses one fixed array per device compiled into the library.
  *   - Calls are asynchronous on `stream`: they enqueue kernels and return without waiting.
  *   - The return value is a status: NVFP4_OK (0) on success.  On a negative status nothing
  *     was enqueued (argument checks run before any launch), except NVFP4_ECUDA, which reports
  *     a failed launch; nvfp4_last_cuda_error() then names the CUDA error.
  *   - Layouts are row-major.  A packed row stores element 2j in the LOW nibble of byte j and
  *     element 2j+1 in the HIGH nibble.  Block scales run along the contiguous dimension.
- *   - The library keeps no global state apart from a per-thread copy of the last CUDA error;
- *     calls on different streams may run concurrently if their workspaces differ.
+ *   - The library keeps no global state apart from a per-thread copy of the last CUDA error
+ *     and the fixed array of moe_nvfp4_forward_static; calls on different streams may run
+ *     concurrently if their workspaces differ.
  */
 #ifndef NVFP4_MOE_H
 #define NVFP4_MOE_H
@@ -173,6 +175,39 @@ NVFP4_API int moe_nvfp4_read_error_flag(const void *workspace, int32_t *host_fla
 NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int64_t E,
                     int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
                     int32_t *error_flag, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- fixed-scratch forward */
+
+/* Largest T*K*I that moe_nvfp4_forward_static takes: its scratch holds T*K rows of I bf16
+ * values (2^18 values = 512 KB; at I = 2048 and K = 8 that is T <= 16). */
+#define NVFP4_STATIC_MAX_H_ELEMS 262144
+
+/* The small-batch forward of moe_nvfp4_forward (its GEMV path: same kernels, same result)
+ * without a caller workspace.  The pages have no counterpart to this call: it exists for
+ * callers that cannot hand the library any device memory, such as a decode loop that has
+ * committed all free memory to its KV-cache pool and holds only the layer's tensors.
+ * Arguments, layouts, alignment and the computed function are those of moe_nvfp4_forward,
+ * except:
+ *   error_flag  [1] int32, may be NULL: receives what the workspace flag of
+ *               moe_nvfp4_forward would (0, bit 0 = an id outside [0, E), bit 1 = a
+ *               device-side wait gave up); overwritten by every call; 4-byte aligned.
+ * Scratch: one array of NVFP4_STATIC_MAX_H_ELEMS bf16 per device, inside the library; no
+ * call allocates or frees memory.  Nothing in it needs to start at zero.  It keeps the last
+ * call's intermediate values after that call ends.  All calls on a device share it, so
+ * calls that can overlap in time (different streams, or different host threads, on the
+ * same device) race; calls on one stream are ordered and safe.  The first call on each
+ * device looks the array's address up (cudaGetSymbolAddress): make that first call before
+ * any stream capture begins on that device.
+ * Errors: EINVAL (null or misaligned pointer, dimension <= 0), ESHAPE (the limits of
+ * moe_nvfp4_forward, T*K*I > NVFP4_STATIC_MAX_H_ELEMS, or a shape the GEMV path does not
+ * take: T*K > 1024, H > 6144 or I > 3072), ECUDA. */
+NVFP4_API int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *topk_ids,
+                                       const float *topk_w, int64_t T, int64_t H, int64_t I,
+                                       int64_t E, int64_t K, const uint8_t *w_gu,
+                                       const uint8_t *s_gu, const float *g_gu,
+                                       const uint8_t *w_dn, const uint8_t *s_dn,
+                                       const float *g_dn, __nv_bfloat16 *out,
+                                       int32_t *error_flag, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

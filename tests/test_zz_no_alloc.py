@@ -1,0 +1,82 @@
+"""moe_nvfp4_forward_static (fixed library scratch, no workspace) against moe_nvfp4_forward.
+
+Both run the GEMV kernels, so the static call must reproduce the workspace call on the same
+inputs; the bar is the MoE tolerance of the parity tests (relative Frobenius error <= 2e-3,
+max abs error <= 1e-2 * max|ref|).  Two calls in a row with different batches check that
+what the first call leaves in the shared scratch does not leak into the second.  This file
+is collected last and needs nothing from the other test files, so it passes alone too."""
+import pytest
+import torch
+
+import synth
+from helpers import MAX_ABS, REL_FRO
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import bit_quantized_moe_nvfp4_b200 as m
+    return m
+
+
+def _layer(nv, E, H, I, seed):
+    gu, dn = synth.expert_weights_bf16(E, H, I, seed, device="cuda")
+    return list(nv.nvfp4_quantize(gu)) + list(nv.nvfp4_quantize(dn))
+
+
+def _close(got, ref):
+    g, r = got.double(), ref.double()
+    nr = torch.linalg.vector_norm(r).item()
+    assert nr > 0.0
+    rel = (torch.linalg.vector_norm(g - r).item()) / nr
+    mab = (g - r).abs().max().item() / r.abs().max().item()
+    assert rel <= REL_FRO, f"relative Frobenius error {rel:.3e} > {REL_FRO}"
+    assert mab <= MAX_ABS, f"max abs error {mab:.3e} * max|ref| > {MAX_ABS}"
+
+
+def _batch(T, E, K, H, seed):
+    x = synth.activations_bf16(T, H, seed).cuda()
+    ids, w = synth.routing(T, E, K, seed, zipf_bias=1.0)
+    return x, ids.cuda(), w.cuda()
+
+
+@pytest.mark.parametrize("shape", [(32, 6144, 2048, 8, [16, 3]), (16, 192, 128, 4, [37, 5])],
+                         ids=["h6144_i2048", "h192_i128"])
+def test_two_calls_match_workspace_forward(nv, shape):
+    E, H, I, K, Ts = shape
+    layer = _layer(nv, E, H, I, seed=11)
+    flag = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    for n, T in enumerate(Ts):
+        x, ids, w = _batch(T, E, K, H, seed=100 + n)
+        got = nv.moe_nvfp4_forward_static(x, ids, w, *layer, error_flag=flag)
+        ref = nv.moe_nvfp4_forward(x, ids, w, *layer, path=nv.PATH_GEMV)
+        torch.cuda.synchronize()
+        _close(got, ref)
+        assert int(flag.item()) == 0
+
+
+def test_bad_id_sets_flag(nv):
+    E, H, I, K, T = 8, 128, 64, 2, 6
+    layer = _layer(nv, E, H, I, seed=3)
+    x, ids, w = _batch(T, E, K, H, seed=4)
+    ids[2, 1] = E + 5
+    flag = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    got = nv.moe_nvfp4_forward_static(x, ids, w, *layer, error_flag=flag)
+    ws = nv.alloc_moe_workspace(T, H, I, E, K)
+    ref = nv.moe_nvfp4_forward(x, ids, w, *layer, workspace=ws, path=nv.PATH_GEMV)
+    _close(got, ref)
+    assert int(flag.item()) == nv.moe_nvfp4_read_error_flag(ws) == 1
+    # the next good call clears it
+    ids[2, 1] = 0
+    nv.moe_nvfp4_forward_static(x, ids, w, *layer, out=got, error_flag=flag)
+    assert int(flag.item()) == 0
+
+
+def test_batch_above_the_fixed_scratch_is_rejected(nv):
+    E, H, I, K = 16, 128, 2048, 8
+    T = 17                                   # 17 * 8 * 2048 > 2^18 bf16 values
+    layer = _layer(nv, E, H, I, seed=5)
+    x, ids, w = _batch(T, E, K, H, seed=6)
+    with pytest.raises(nv.NVFP4Error, match="ESHAPE"):
+        nv.moe_nvfp4_forward_static(x, ids, w, *layer)
