@@ -12,11 +12,12 @@
 //            y[slot, n] = w[pair] * g_dn * D
 //   combine (combine.cu): out[t] = bf16( sum over k of y[slot(t, k)] )
 //
-// One persistent CTA per SM walks the tiles (expert, 224-slot n-tile, 128-row m-tile) with
+// One persistent CTA per SM walks the tiles (expert, 192-slot n-tile, 128-row m-tile) with
 // warp-specialised roles:
-//   warp 0     TMA producer: packed weight rows (2 boxes of 64 rows x 32 bytes) and the
-//              activation tile (224 rows x 64 elements, 128-byte swizzle) per 64-wide K step;
-//   warp 1     allocates TMEM and issues tcgen05.mma (M=128, N<=224, K=16, fp32 in TMEM)
+//   warp 0     TMA producer: packed weight rows (2 boxes of 64 rows x 64 bytes) and the
+//              activation tile (2 boxes of 192 rows x 64 elements, 128-byte swizzle) per
+//              128-wide K step, into a 3-stage ring;
+//   warp 1     allocates TMEM and issues tcgen05.mma (M=128, N<=192, K=16, fp32 in TMEM)
 //              with the weight operand read from TMEM and the activations from shared memory;
 //   warps 2-9  dequantize: half a weight row per thread, E2M1 x E4M3 -> f16 (gate/up) or
 //              bf16 (down), exact either way (at most 6 significant bits), stored straight
@@ -24,7 +25,7 @@
 //              touches shared memory;
 //   warps 10-13 epilogue: tcgen05.ld of the accumulator, global scale, SwiGLU or routing
 //              weight, stores.
-// Accumulators are double-buffered in TMEM (2 x 224 columns, next to two 32-column weight
+// Accumulators are double-buffered in TMEM (2 x 192 columns, next to two 64-column weight
 // operand slots), so the epilogue of one tile overlaps the main loop of the next.  The weights sit on M ("swap AB") because experts get
 // anywhere from 0 to thousands of tokens: the token count only changes N.
 #include <cuda.h>
@@ -36,12 +37,14 @@ namespace nvfp4 {
 
 namespace {
 
-// Pipeline depth and dequant width (compile-time tunables; defaults measured on B200).
+// Pipeline depth, tile sizes and dequant width (compile-time tunables; defaults measured on
+// B200: a 128-wide K step issues 8 MMAs per barrier round trip, which is what lets the
+// single issuing thread keep the tensor pipe busy).
 #ifndef NVFP4_GEMM_STAGES
-#define NVFP4_GEMM_STAGES 6
+#define NVFP4_GEMM_STAGES 3
 #endif
 #ifndef NVFP4_GEMM_BN
-#define NVFP4_GEMM_BN 224
+#define NVFP4_GEMM_BN 192
 #endif
 #ifndef NVFP4_GEMM_A_SLOTS
 #define NVFP4_GEMM_A_SLOTS 2
@@ -49,9 +52,14 @@ namespace {
 #ifndef NVFP4_GEMM_DEQUANT_WARPS
 #define NVFP4_GEMM_DEQUANT_WARPS 8
 #endif
+#ifndef NVFP4_GEMM_BK
+#define NVFP4_GEMM_BK 128
+#endif
 constexpr int BM = 128;          // weight rows per tile (TMEM lanes)
 constexpr int BN = NVFP4_GEMM_BN;   // token slots per tile (MMA N, multiple of 16)
-constexpr int BK = 64;           // reduction elements per stage
+constexpr int BK = NVFP4_GEMM_BK;   // reduction elements per stage (64 or 128)
+constexpr int kBoxes = BK / 64;     // 64-element (128-byte) activation boxes per stage
+static_assert(BK == 64 || BK == 128, "BK: 64 or 128");
 constexpr int kS = NVFP4_GEMM_STAGES;           // stages: packed weights + activation tile
 constexpr int kSA = NVFP4_GEMM_A_SLOTS;         // weight operand slots in TMEM
 constexpr int kDQW = NVFP4_GEMM_DEQUANT_WARPS;  // 4 (full rows) or 8 (half rows)
@@ -60,15 +68,17 @@ constexpr int kThreads = 32 * (kWarpEpi + 4);
 static_assert(kDQW == 4 || kDQW == 8, "dequant warps: 4 or 8");
 
 // Tensor memory: two fp32 accumulators of BN columns, then kSA weight operands of BK/2
-// columns (64 16-bit values of a row per lane) -- 2*224 + 2*32 = 512 columns.
+// columns (BK 16-bit values of a row per lane) -- 2*192 + 2*64 = 512 columns.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemA = 2 * BN;
 constexpr uint32_t kACols = BK / 2;
 static_assert(kTmemA + kSA * kACols <= kTmemCols, "TMEM budget");
 
-constexpr uint32_t kBBytes = BN * BK * 2;     // activation tile (128-byte swizzle)
-static_assert(kBBytes % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
-constexpr uint32_t kPBytes = BM * BK / 2;     // 4 KB packed weights
+constexpr uint32_t kBoxBytes = BN * 128;     // one 64-element activation box (128-byte swizzle)
+constexpr uint32_t kBBytes = kBoxes * kBoxBytes;
+static_assert(kBoxBytes % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
+constexpr uint32_t kPBytes = BM * BK / 2;     // packed weights (4 or 8 KB)
+constexpr int kSB = BK / 16;                  // block-scale bytes per row per stage
 constexpr uint32_t kSmemB = 0;
 constexpr uint32_t kSmemP = kSmemB + kS * kBBytes;
 constexpr uint32_t kSmemBars = kSmemP + kS * kPBytes;
@@ -212,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();   // routing tables (and the activations) come from earlier kernels
   const int n_act = *a.n_active;
   const int total_tiles = n_act > 0 ? a.tile_prefix[n_act] * p.m_tiles : 0;
-  const int kblocks = p.K / BK;
+  const int kblocks = (p.K + BK - 1) / BK;   // a last half stage (K % 128 == 64) reads zeros
   const int64_t I = a.I, H = a.H;
 
   // Bounded wait; after any wait of the CTA has given up, later slow waits return at once.
@@ -247,7 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           unsigned char *pk = smem + kSmemP + s * kPBytes;
           tma_load_2d(pk, &tmap_w, kb * (BK / 2), row0, &full[s]);
           tma_load_2d(pk + 64 * (BK / 2), &tmap_w, kb * (BK / 2), row1, &full[s]);
-          tma_load_2d(smem + kSmemB + s * kBBytes, &tmap_b, kb * BK, t.slot0, &full[s]);
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_2d(smem + kSmemB + s * kBBytes + bx * kBoxBytes, &tmap_b, kb * BK + 64 * bx,
+                        t.slot0, &full[s]);
         }
         if (*(volatile int *)abort) break;
       }
@@ -274,8 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t a_tmem = tmem_base + kTmemA + sa * kACols;
             const uint64_t db = smem_desc_sw128(smem_u32(smem + kSmemB + s * kBBytes));
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)   // K=16: 8 TMEM columns, 32 bytes of B
-              umma_ts(d_tmem, a_tmem + 8 * kk, db + 2 * kk, idesc, kb > 0 || kk > 0);
+            for (int kk = 0; kk < BK / 16; ++kk)   // K=16: 8 TMEM columns, 32 bytes of a B box
+              umma_ts(d_tmem, a_tmem + 8 * kk,
+                      db + (uint64_t)((kk / 4) * (kBoxBytes >> 4) + 2 * (kk % 4)), idesc,
+                      kb > 0 || kk > 0);
           }
           umma_commit(&freeb[s]);
           umma_commit(&afree[sa]);
@@ -288,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warp w writes TMEM lanes 32*(w%4)..+31: lane L holds weight-operand row L.  With 8
     // warps, the second four write the upper half of each row's 64 elements.
     constexpr int kPerRow = kDQW / 4;            // threads per row (1 or 2)
-    constexpr int NW = 8 / kPerRow;              // packed words per thread per step
+    constexpr int NW = BK / 8 / kPerRow;         // packed words per thread per step
+    static_assert(NW == 4 || NW == 8, "one tcgen05.st of 16 or 32 columns per step");
     const int q = warp & 3;
     const int part = (warp - 2) / 4;             // 0, or 1 for the second four warps
     const int L = q * 32 + lane;                 // operand row = TMEM lane
@@ -308,27 +324,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         prow = L;
         wrow = (int64_t)t.e * H + n;
       }
-      // Block scales of this row: 4 bytes per K step, fetched 16 bytes (four steps) at a
-      // time, two groups ahead.  Rows whose scale run is not 16-byte aligned take 4-byte loads.
+      // Block scales of this row: BK/16 bytes per K step (one or two 32-bit words), fetched
+      // 16 bytes at a time, two groups ahead.  Rows whose scale run is not 16-byte aligned
+      // take 4-byte loads; words past the end of the row read as 0.
+      constexpr int kWS = kSB / 4;             // scale words per stage
+      constexpr int kSPG = 4 / kWS;            // stages per 16-byte group
       const uint8_t *srow = p.scales + wrow * (p.K / 16);
+      const int n_words = p.K / 64;
       const bool wide = (p.K % 256) == 0;
       auto group = [&](int g) -> uint4 {
-        if (!valid || 4 * g >= kblocks) return make_uint4(0, 0, 0, 0);
+        if (!valid || 4 * g >= n_words) return make_uint4(0, 0, 0, 0);
         if (wide) return __ldg(reinterpret_cast<const uint4 *>(srow) + g);
         const uint32_t *w = reinterpret_cast<const uint32_t *>(srow) + 4 * g;
-        const int left = kblocks - 4 * g;
+        const int left = n_words - 4 * g;
         return make_uint4(__ldg(w), left > 1 ? __ldg(w + 1) : 0u, left > 2 ? __ldg(w + 2) : 0u,
                           left > 3 ? __ldg(w + 3) : 0u);
       };
       uint4 g0 = group(0), g1 = group(1), g2 = group(2);
       for (int kb = 0; kb < kblocks; ++kb, ++kg) {
         const int s = kg % kS, sa = kg % kSA;
-        if (kb > 0 && (kb & 3) == 0) {
+        if (kb > 0 && kb % kSPG == 0) {
           g0 = g1;
           g1 = g2;
-          g2 = group((kb >> 2) + 2);
+          g2 = group(kb / kSPG + 2);
         }
-        const int w4 = kb & 3;
+        const int w4 = (kb % kSPG) * kWS + (kWS == 2 ? part : 0);
         const uint32_t sc = w4 == 0 ? g0.x : (w4 == 1 ? g0.y : (w4 == 2 ? g0.z : g0.w));
         bool ok = wait(&full[s], (kg / kS) & 1);
         if (kg >= kSA) ok = wait(&afree[sa], ((kg / kSA) - 1) & 1) && ok;
@@ -347,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!valid || !ok)
 #pragma unroll
           for (int i = 0; i < NW; ++i) w[i] = 0u;
-        const uint32_t scp = sc >> (8 * (NW / 2) * part);    // this part's block scales
+        const uint32_t scp = kWS == 2 ? sc : sc >> (8 * (NW / 2) * part);   // this part's scales
         uint32_t o[4 * NW];
         if (p.mode == 0)
           dequant_words<true, NW>(w, scp, o);
@@ -517,7 +537,7 @@ int launch_gemm(const MoeArgs &a, int mode, cudaStream_t s) {
   const uint64_t brows = (uint64_t)(a.T * a.K + kGatherPadRows);
   if (make_map(&tb, mode == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                2, mode == 0 ? (const void *)a.xs : (const void *)a.h,
-               (uint64_t)p.K, brows, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+               (uint64_t)p.K, brows, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return NVFP4_ECUDA;
   cudaError_t e =
       cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
