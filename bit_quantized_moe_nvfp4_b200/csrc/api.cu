@@ -157,13 +157,15 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   if (path == NVFP4_PATH_GEMV && !gemv_supported(T, H, I, K)) return NVFP4_ESHAPE;
 
   if (path == NVFP4_PATH_GEMV) {
-    // two kernels: routing is recomputed inside each, the combine is fused into the second
+    // routing is recomputed inside each projection kernel, so there is no route launch
     if (int s = record(ev, 0, stream)) return s;
     if (int s = record(ev, 1, stream)) return s;
     if (int s = launch_gemv_gateup(a, stream)) return s;
     if (int s = record(ev, 2, stream)) return s;
     if (int s = launch_gemv_down(a, stream)) return s;
     if (int s = record(ev, 3, stream)) return s;
+    if (!gemv_fused_combine(T))
+      if (int s = launch_combine_pairs(a, stream)) return s;
     return record(ev, 4, stream);
   }
 

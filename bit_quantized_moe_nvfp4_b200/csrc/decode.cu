@@ -39,17 +39,21 @@ namespace {
 #define NVFP4_GEMV_PAIRS 4
 #endif
 #ifndef NVFP4_GEMV_DOWN_ROWS
-#define NVFP4_GEMV_DOWN_ROWS 8
+#define NVFP4_GEMV_DOWN_ROWS 32
 #endif
 #ifndef NVFP4_GEMV_CTAS_PER_SM
 #define NVFP4_GEMV_CTAS_PER_SM 3
 #endif
+#ifndef NVFP4_GEMV_DOWN_STAGES
+#define NVFP4_GEMV_DOWN_STAGES NVFP4_GEMV_STAGES
+#endif
 #ifndef NVFP4_GEMV_DOWN_CTAS_PER_SM
-#define NVFP4_GEMV_DOWN_CTAS_PER_SM 4
+#define NVFP4_GEMV_DOWN_CTAS_PER_SM 2
 #endif
 constexpr int kStages = NVFP4_GEMV_STAGES;       // shared-memory ring depth
 constexpr int kPairs = NVFP4_GEMV_PAIRS;         // gate/up row pairs per stage
 constexpr int kDownRows = NVFP4_GEMV_DOWN_ROWS;  // rows per stage (down kernel)
+constexpr int kDownStages = NVFP4_GEMV_DOWN_STAGES;
 constexpr int kMaxConsumerWarps = 6;
 constexpr int64_t kGemvMaxPairs = 1024;  // T*K handled by the GEMV path
 
@@ -593,6 +597,365 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 3 : 1)
   }
 }
 
+// ================================================================== projections on mma.sync
+// Both projections of the GEMV path run on the tensor cores with mma.sync.m16n8k16
+// (f16 x f16 -> fp32): M = 16 weight rows of one expert, N = 8 token slots, K = 16.
+//   MODE 0, gate/up: rows = gate rows j..j+7 and up rows j..j+7; the activations are x;
+//           result h[slot, j+r] = bf16( silu(g_gu * gate_r) * g_gu * up_r )  (SwiGLU)
+//   MODE 1, down:    rows = output rows r0..r0+15; the activations are the h rows of the
+//           expert's slots; result y[pair, r0+r] = w[pair] * g_dn * (W_dn h)_r, combined
+//           over k afterwards (combine.cu)
+// A unit is one such 16-row tile; each CTA takes a contiguous range of units in expert
+// order, so an expert's activations are loaded once per CTA.  Since a dot product may sum its terms in any order, the K index of the MMA is
+// mapped to memory so that each lane decodes only contiguous bytes: lane (g, t) (g = lane/4,
+// t = lane%4) owns elements 32t..32t+31 of every 128-element chunk, for weight rows g and
+// g+8 (A operand) and for token g (B operand); MMA i of a chunk takes elements
+// 32t+4i..32t+4i+3 of each lane.  E2M1 codes become f16 with the hardware convert and are
+// multiplied by their E4M3 block scale in f16 (exact: at most 6 significant bits), the
+// activations are f16 with the per-token power-of-two scale, and the tensor core sums in
+// fp32.  This takes about a third of the instructions of a CUDA-core dot product per byte.
+constexpr int kGuWarps = 16;                  // compute warps
+constexpr int kGuMaxChunks = 3;               // 128-element chunks per warp: H <= 6144
+constexpr int kGuTok = 8;                     // token slots per group (MMA N)
+constexpr int kGuRedFloats = kGuWarps * 16 * kGuTok + 2 * kGuTok;   // per reduction slot
+
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
+  return *reinterpret_cast<uint32_t *>(&r);
+}
+
+struct GuSmem {
+  uint32_t bars, stages, red, smax, ids, act_e, act_off, misc, hist, total;
+};
+
+__host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, int n, int E) {
+  GuSmem s;
+  uint32_t o = 0;
+  s.bars = o;
+  o += 8 * (2 * S + 2 * kRedSlots);
+  o = align_up(o, 128);
+  s.stages = o;
+  o += stage_bytes * S;
+  s.red = o;
+  o += 4 * kRedSlots * kGuRedFloats;
+  s.smax = o;
+  o += 4 * kGuWarps * kGuTok;
+  s.ids = o;
+  o += 4 * n;
+  const int na = min(E, n);
+  s.act_e = o;
+  o += 4 * na;
+  s.act_off = o;
+  o += 4 * (na + 1);
+  s.misc = o;
+  o += 16;
+  s.hist = o;
+  o += 4 * E;
+  s.total = align_up(o, 128);
+  return s;
+}
+
+// Stage geometry for a reduction length Kd: 16 packed rows at a stride of Kd/2 + 16 bytes
+// (the pad spreads the rows over the shared-memory banks), then the block-scale runs of rows
+// 0..7 and 8..15.
+__host__ __device__ inline uint32_t gu_row_stride(int64_t Kd) { return (uint32_t)(Kd / 2 + 16); }
+__host__ __device__ inline uint32_t gu_stage_bytes(int64_t Kd) {
+  return 16 * gu_row_stride(Kd) + 2 * span_bytes(8 * (Kd / 16));
+}
+
+// blockDim = 32 * (kGuWarps + 2): warp 0 produces, warps 1..kGuWarps compute, the last warp
+// finalizes.
+template <int MODE, int S>
+__global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
+    gemv_mma_kernel(MoeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_abort;
+  constexpr int CW = kGuWarps;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t H = a.H, I = a.I, K = a.K;
+  const int64_t Kd = MODE == 0 ? H : I;          // reduction length
+  const int n = (int)(a.T * K);
+  const int E = (int)a.E;
+  const uint32_t rstride = gu_row_stride(Kd), stage_bytes = gu_stage_bytes(Kd);
+  const GuSmem L = gu_smem_layout(S, stage_bytes, n, E);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
+  uint64_t *empty = full + S;
+  uint64_t *rfull = empty + S;
+  uint64_t *rfree = rfull + kRedSlots;
+  unsigned char *stage_base = smem + L.stages;
+  float *red = reinterpret_cast<float *>(smem + L.red);
+  float *smax = reinterpret_cast<float *>(smem + L.smax);
+  CtaRoute R{reinterpret_cast<int *>(smem + L.ids), reinterpret_cast<int *>(smem + L.act_e),
+             reinterpret_cast<int *>(smem + L.act_off), reinterpret_cast<int *>(smem + L.misc)};
+  int *hist = reinterpret_cast<int *>(smem + L.hist);
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], CW);
+    }
+    for (int s = 0; s < kRedSlots; ++s) {
+      mbar_init(&rfull[s], CW);
+      mbar_init(&rfree[s], 1);
+    }
+    mbar_init_fence();
+  }
+  if (MODE == 0) pdl_wait();   // x and the ids come from earlier kernels
+  // (MODE 1: the ids were complete before the gate/up kernel let this grid start, so the
+  // routing and the weight stream start before griddepcontrol.wait)
+  const bool bad = cta_route(a.ids, n, E, R, hist);
+  if (MODE == 0 && blockIdx.x == 0 && threadIdx.x == 0 && a.flag) *a.flag = bad ? kFlagBadId : 0;
+  pdl_launch_dependents();  // the next kernel may start its prologue
+
+  const int n_act = *R.n_act;
+  const int64_t upe = MODE == 0 ? I / 8 : H / 16;   // units per expert
+  const int64_t units = (int64_t)n_act * upe;
+  const int64_t U0 = units * blockIdx.x / gridDim.x, U1 = units * (blockIdx.x + 1) / gridDim.x;
+  const uint32_t rowb = (uint32_t)(Kd / 2), sclb = (uint32_t)(Kd / 16);
+  const uint32_t scl_off = 16 * rstride;
+  const uint32_t span_stride = span_bytes(8 * sclb);
+
+  if (warp == 0) {
+    // ------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      for (int64_t u = U0; u < U1; ++u, ++s) {
+        const int ai = (int)(u / upe);
+        const int e = R.act_e[ai];
+        const int idx = s % S;
+        if (s >= S && (*(volatile int *)&s_abort || !mbar_wait(&empty[idx], ((s / S) - 1) & 1))) {
+          if (!*(volatile int *)&s_abort) report_timeout(a.flag);
+          *(volatile int *)&s_abort = 1;
+          break;
+        }
+        unsigned char *st = stage_base + (size_t)idx * stage_bytes;
+        // rows 0..7 and 8..15 of the tile, as row indices inside the expert's weight block
+        const int64_t lr0 = MODE == 0 ? (u % upe) * 8 : (u % upe) * 16;
+        const int64_t lr1 = MODE == 0 ? I + lr0 : lr0 + 8;
+        const int64_t rows_pe = MODE == 0 ? 2 * I : H;
+        const uint8_t *wblock = (MODE == 0 ? a.w_gu : a.w_dn) + (int64_t)e * rows_pe * rowb;
+        const uint8_t *sblock = (MODE == 0 ? a.s_gu : a.s_dn) + (int64_t)e * rows_pe * sclb;
+        const int64_t lg = lr0 * sclb, lu = lr1 * sclb;
+        const uint32_t span_g = (uint32_t)(((lg + 8 * sclb + 15) & ~15ll) - (lg & ~15ll));
+        const uint32_t span_u = (uint32_t)(((lu + 8 * sclb + 15) & ~15ll) - (lu & ~15ll));
+        mbar_arrive_expect_tx(&full[idx], 16u * rowb + span_g + span_u);
+#pragma unroll 1
+        for (int r = 0; r < 8; ++r) {
+          bulk_g2s(st + r * rstride, wblock + (lr0 + r) * rowb, rowb, &full[idx]);
+          bulk_g2s(st + (8 + r) * rstride, wblock + (lr1 + r) * rowb, rowb, &full[idx]);
+        }
+        bulk_g2s_span(st + scl_off, sblock, lg, 8 * sclb, &full[idx]);
+        bulk_g2s_span(st + scl_off + span_stride, sblock, lu, 8 * sclb, &full[idx]);
+      }
+      const int issued = s;
+      for (int t = max(0, issued - S); t < issued; ++t)
+        if (!mbar_wait(&full[t % S], (t / S) & 1)) report_timeout(a.flag);
+    }
+    return;
+  }
+
+  if (warp == CW + 1) {
+    // ------------------------------------------------ finalizer
+    int it = 0, cur_a = -1, slot0 = 0, cnt = 0;
+    float gsc = 0.f;
+    for (int64_t u = U0; u < U1; ++u) {
+      const int ai = (int)(u / upe);
+      const int64_t j = MODE == 0 ? (u % upe) * 8 : (u % upe) * 16;   // first row / pair
+      if (ai != cur_a) {
+        cur_a = ai;
+        slot0 = R.act_off[ai];
+        cnt = R.act_off[ai + 1] - slot0;
+        gsc = __ldg((MODE == 0 ? a.g_gu : a.g_dn) + R.act_e[ai]);
+      }
+      for (int grp = 0; grp * kGuTok < cnt; ++grp, ++it) {
+        const int nt = min(kGuTok, cnt - grp * kGuTok);
+        const int sl = it % kRedSlots;
+        const bool ok = warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag);
+        const float *rb = red + (size_t)sl * kGuRedFloats;
+        if (MODE == 0) {
+          for (int q = lane; ok && q < 8 * nt; q += 32) {
+            const int tk = q >> 3, r = q & 7;   // token slot of the group, row pair
+            float gs = 0.f, us = 0.f;
+#pragma unroll 4
+            for (int w = 0; w < CW; ++w) {
+              gs += rb[w * 128 + r * 8 + tk];
+              us += rb[w * 128 + (8 + r) * 8 + tk];
+            }
+            const float ps = rb[CW * 128 + tk];
+            const float gate = gs * gsc * ps, up = us * gsc * ps;
+            const int slot = slot0 + grp * kGuTok + tk;
+            a.h[(int64_t)slot * I + j + r] = __float2bfloat16_rn(silu_f32(gate) * up);
+          }
+        } else {
+          for (int q = lane; ok && q < 16 * nt; q += 32) {
+            const int tk = q >> 4, r = q & 15;  // token slot of the group, output row
+            float ys = 0.f;
+#pragma unroll 4
+            for (int w = 0; w < CW; ++w) ys += rb[w * 128 + r * 8 + tk];
+            const float ps = rb[CW * 128 + tk];
+            const int pair = __float_as_int(rb[CW * 128 + kGuTok + tk]);
+            a.y[(int64_t)pair * H + j + r] = ys * gsc * ps * __ldg(a.w + pair);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfree[sl]);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------ compute warps
+  if (MODE == 1) pdl_wait();   // h is written by the gate/up kernel
+  const int cw = warp - 1;
+  const int g = lane >> 2, t = lane & 3;
+  const int nchunk = (int)((Kd + 127) / 128);
+  const int nthreads_c = CW * 32;
+  uint32_t xr[kGuMaxChunks][16];     // token g's activations (f16x2), chunk cw + CW*m
+  float pscale = 1.f;                // 2^-p of token g
+  int loaded_tok = -2;               // activation row that lane group g holds
+  int mypair = -1;                   // pair of slot g of the current group
+  const __nv_bfloat16 *arow = MODE == 0 ? a.x : a.h;
+#pragma unroll
+  for (int m = 0; m < kGuMaxChunks; ++m)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xr[m][i] = 0u;
+  int cur_a = -1, ngroups = 0, cnt = 0;
+  int s = 0, it = 0;
+  for (int64_t u = U0; u < U1; ++u, ++s) {
+    const int ai = (int)(u / upe);
+    const int64_t lr0 = MODE == 0 ? (u % upe) * 8 : (u % upe) * 16;
+    const int64_t lr1 = MODE == 0 ? I + lr0 : lr0 + 8;
+    const int idx = s % S;
+    const bool new_expert = ai != cur_a;
+    if (new_expert) {
+      cur_a = ai;
+      cnt = R.act_off[ai + 1] - R.act_off[ai];
+      ngroups = (cnt + kGuTok - 1) / kGuTok;
+    }
+    const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
+    const unsigned char *st = stage_base + (size_t)idx * stage_bytes;
+    const unsigned char *sgb = st + scl_off + ((lr0 * sclb) & 15);
+    const unsigned char *sub = st + scl_off + span_stride + ((lr1 * sclb) & 15);
+    for (int grp = 0; grp < ngroups; ++grp, ++it) {
+      const int nt = min(kGuTok, cnt - grp * kGuTok);
+      const bool last = grp == ngroups - 1;
+      if (ngroups > 1 || new_expert) {
+        // token of slot g of this group; the decision to reload depends only on shared
+        // data, so all compute warps take it together
+        const int pr = pairs_of_expert<kGuTok>(R.ids, n, R.act_e[ai], grp * kGuTok, lane);
+        mypair = __shfl_sync(0xFFFFFFFFu, pr, g & 7);
+        // activation row of slot g: token (gate/up) or h row of the slot (down)
+        const int tok = g >= nt ? -1
+                        : (MODE == 0 ? (int)(mypair / K) : R.act_off[ai] + grp * kGuTok + g);
+        const bool reload = __any_sync(0xFFFFFFFFu, tok != loaded_tok);
+        if (reload) {
+          loaded_tok = tok;
+          // pass 1: largest magnitude of token g over the whole row (all compute warps)
+          float mx = 0.f;
+          if (tok >= 0) {
+#pragma unroll
+            for (int m = 0; m < kGuMaxChunks; ++m) {
+              const int c = cw + CW * m;
+              if (c < nchunk && c * 128 + 32 * t < Kd) {
+                uint4 v[4];
+                mx = fmaxf(mx, load_bf16x32(arow + (int64_t)tok * Kd + c * 128 + 32 * t, v));
+              }
+            }
+          }
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+          if (t == 0) smax[cw * kGuTok + g] = mx;
+          named_sync(1, nthreads_c);
+          float mm = 0.f;
+          for (int w = 0; w < CW; ++w) mm = fmaxf(mm, smax[w * kGuTok + g]);
+          const int p = prescale_exponent(mm);
+          pscale = exp2i(-p);
+          const float sp = exp2i(p);
+#pragma unroll
+          for (int m = 0; m < kGuMaxChunks; ++m) {
+            const int c = cw + CW * m;
+            if (tok >= 0 && c < nchunk && c * 128 + 32 * t < Kd) {
+              uint4 v[4];
+              load_bf16x32(arow + (int64_t)tok * Kd + c * 128 + 32 * t, v);
+              to_f16x32(v, sp, xr[m]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) xr[m][i] = 0u;
+            }
+          }
+          named_sync(1, nthreads_c);   // smax is rewritten by the next reload
+        }
+      }
+      // partial dot products over this warp's chunks: d[0..3] = rows (g, g+8) x tokens
+      // (2t, 2t+1) as the m16n8 accumulator layout has them; two chains for latency
+      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (have) {
+#pragma unroll
+        for (int m = 0; m < kGuMaxChunks; ++m) {
+          const int c = cw + CW * m;
+          if (c >= nchunk) break;
+          const bool lv = c * 128 + 32 * t < Kd;
+          uint4 wg = make_uint4(0u, 0u, 0u, 0u), wu = wg;
+          uint32_t sg = 0u, su = 0u;
+          if (lv) {
+            wg = *reinterpret_cast<const uint4 *>(st + g * rstride + c * 64 + 16 * t);
+            wu = *reinterpret_cast<const uint4 *>(st + (8 + g) * rstride + c * 64 + 16 * t);
+            sg = *reinterpret_cast<const unsigned short *>(sgb + g * sclb + c * 8 + 2 * t);
+            su = *reinterpret_cast<const unsigned short *>(sub + g * sclb + c * 8 + 2 * t);
+          }
+          // block scales as f16 pairs: blocks 2t (elements 0..15 of the lane) and 2t+1
+          const uint32_t sgh = e4m3x2_to_f16x2(sg), suh = e4m3x2_to_f16x2(su);
+          const uint32_t Sg[2] = {__byte_perm(sgh, 0, 0x1010), __byte_perm(sgh, 0, 0x3232)};
+          const uint32_t Su[2] = {__byte_perm(suh, 0, 0x1010), __byte_perm(suh, 0, 0x3232)};
+          const uint32_t wgw[4] = {wg.x, wg.y, wg.z, wg.w};
+          const uint32_t wuw[4] = {wu.x, wu.y, wu.z, wu.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {            // word q: elements 8q..8q+7, MMAs 2q, 2q+1
+            uint32_t hg[4], hu[4];
+            e2m1x8_to_f16x2x4(wgw[q], hg);
+            e2m1x8_to_f16x2x4(wuw[q], hu);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              hg[k] = hmul2_u32(hg[k], Sg[q >> 1]);
+              hu[k] = hmul2_u32(hu[k], Su[q >> 1]);
+            }
+            // MMA 2q: elements 8q..8q+3; MMA 2q+1: elements 8q+4..8q+7
+            mma_16816_f16(d0, hg[0], hu[0], hg[1], hu[1], xr[m][4 * q], xr[m][4 * q + 1]);
+            mma_16816_f16(d1, hg[2], hu[2], hg[3], hu[3], xr[m][4 * q + 2], xr[m][4 * q + 3]);
+          }
+        }
+      }
+      if (last) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[idx]);   // this warp is done reading the stage
+      }
+      const int sl = it % kRedSlots;
+      if (it >= kRedSlots) warp_wait(&rfree[sl], ((it / kRedSlots) - 1) & 1, &s_abort, a.flag);
+      float *rb = red + (size_t)sl * kGuRedFloats + cw * 128;
+      *reinterpret_cast<float2 *>(rb + g * 8 + 2 * t) = make_float2(d0[0] + d1[0], d0[1] + d1[1]);
+      *reinterpret_cast<float2 *>(rb + (8 + g) * 8 + 2 * t) =
+          make_float2(d0[2] + d1[2], d0[3] + d1[3]);
+      if (cw == 0 && t == 0) {
+        red[(size_t)sl * kGuRedFloats + CW * 128 + g] = pscale;
+        red[(size_t)sl * kGuRedFloats + CW * 128 + kGuTok + g] = __int_as_float(mypair);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfull[sl]);
+    }
+  }
+}
+
 // ================================================================== down + combine
 // CTA c owns output rows [n0, n0 + nb) for every active expert.  Warp 0 produces, warps
 // 1..CW compute with lanes owning 16 consecutive elements (8 packed bytes, 1 block scale),
@@ -861,8 +1224,6 @@ int resident_blocks(Kern k, int threads, size_t smem) {
   return nb;
 }
 
-int tokens_per_group(int64_t T) { return T <= 1 ? 1 : (T <= 16 ? 2 : 4); }
-
 template <int NT, int P, int S>
 int launch_gateup_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
   const int CW = (int)ceil_div(a.H, 1024);
@@ -874,6 +1235,25 @@ int launch_gateup_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
   if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
   return launch_pdl(gemv_gateup_kernel<NT, P, S>, dim3(num_sms() * min(ctas_per_sm, fit)),
                     dim3(32 * (CW + 2)), L.total, s, a, stage_bytes);
+}
+
+template <int MODE, int S>
+int launch_mma_cfg(const MoeArgs &a, cudaStream_t s) {
+  const int n = (int)(a.T * a.K);
+  const GuSmem L = gu_smem_layout(S, gu_stage_bytes(MODE == 0 ? a.H : a.I), n, (int)a.E);
+  const int fit = resident_blocks(gemv_mma_kernel<MODE, S>, 32 * (kGuWarps + 2), L.total);
+  if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
+  return launch_pdl(gemv_mma_kernel<MODE, S>, dim3(num_sms()), dim3(32 * (kGuWarps + 2)),
+                    L.total, s, a);
+}
+
+// Three stages when they fit in shared memory, else two.
+template <int MODE>
+int launch_mma(const MoeArgs &a, cudaStream_t s) {
+  const int n = (int)(a.T * a.K);
+  const uint32_t sb = gu_stage_bytes(MODE == 0 ? a.H : a.I);
+  if (gu_smem_layout(3, sb, n, (int)a.E).total <= 227u * 1024u) return launch_mma_cfg<MODE, 3>(a, s);
+  return launch_mma_cfg<MODE, 2>(a, s);
 }
 
 template <int NT, int RD, int S>
@@ -897,23 +1277,28 @@ int launch_down_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
 }  // namespace
 
 bool gemv_supported(int64_t T, int64_t H, int64_t I, int64_t K) {
-  return T * K <= kGemvMaxPairs && H <= 1024 * kMaxConsumerWarps && I <= 512 * kMaxConsumerWarps;
+  if (T * K > kGemvMaxPairs) return false;
+  if (T == 1)   // CUDA-core kernels: 32 (gate/up) or 16 (down) elements per lane, 6 warps
+    return H <= 1024 * kMaxConsumerWarps && I <= 512 * kMaxConsumerWarps;
+  const int64_t max_k = (int64_t)kGuWarps * kGuMaxChunks * 128;   // mma kernels
+  return H <= max_k && I <= max_k;
 }
 
+// One token: the CUDA-core kernels (the combine is fused into the down kernel).  More
+// tokens: the mma.sync kernels, which serve up to 8 tokens of an expert per MMA, and a
+// separate combine.
+bool gemv_fused_combine(int64_t T) { return T == 1; }
+
 int launch_gemv_gateup(const MoeArgs &a, cudaStream_t s) {
-  switch (tokens_per_group(a.T)) {
-    case 1: return launch_gateup_cfg<1, kPairs, kStages>(a, s, NVFP4_GEMV_CTAS_PER_SM);
-    case 2: return launch_gateup_cfg<2, kPairs, kStages>(a, s, NVFP4_GEMV_CTAS_PER_SM);
-    default: return launch_gateup_cfg<4, kPairs, kStages>(a, s, 2);
-  }
+  if (gemv_fused_combine(a.T))
+    return launch_gateup_cfg<1, kPairs, kStages>(a, s, NVFP4_GEMV_CTAS_PER_SM);
+  return launch_mma<0>(a, s);
 }
 
 int launch_gemv_down(const MoeArgs &a, cudaStream_t s) {
-  switch (tokens_per_group(a.T)) {
-    case 1: return launch_down_cfg<1, kDownRows, kStages>(a, s, NVFP4_GEMV_DOWN_CTAS_PER_SM);
-    case 2: return launch_down_cfg<2, kDownRows, kStages>(a, s, NVFP4_GEMV_DOWN_CTAS_PER_SM);
-    default: return launch_down_cfg<4, kDownRows, kStages>(a, s, 3);
-  }
+  if (gemv_fused_combine(a.T))
+    return launch_down_cfg<1, kDownRows, kDownStages>(a, s, NVFP4_GEMV_DOWN_CTAS_PER_SM);
+  return launch_mma<1>(a, s);
 }
 
 }  // namespace nvfp4

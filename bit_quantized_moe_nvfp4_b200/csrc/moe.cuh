@@ -46,8 +46,10 @@ constexpr int kGatherPadRows = 256;
 bool gemv_supported(int64_t T, int64_t H, int64_t I, int64_t K);
 int launch_gemv_gateup(const MoeArgs &a, cudaStream_t s);
 int launch_gemv_down(const MoeArgs &a, cudaStream_t s);
+bool gemv_fused_combine(int64_t T);   // the GEMV down kernel also combines (no combine launch)
 // combine of the GEMM path (combine.cu)
 int launch_combine(const MoeArgs &a, cudaStream_t s);
+int launch_combine_pairs(const MoeArgs &a, cudaStream_t s);   // y indexed by pair (GEMV path)
 // GEMM path (gemm.cu)
 int launch_gemm_gateup(const MoeArgs &a, cudaStream_t s);   // gather + gate/up + SwiGLU
 int launch_gemm_down(const MoeArgs &a, cudaStream_t s);

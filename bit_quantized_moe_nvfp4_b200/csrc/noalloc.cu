@@ -7,10 +7,12 @@
 // holds only the layer's own tensors, so it can neither allocate a workspace nor carve one
 // out of a buffer it owns.  The kernels are the ones moe_nvfp4_forward runs on its GEMV
 // path; only the scratch they write differs:
-//   h   [T*K, I] bf16   SwiGLU outputs, one row per routed pair    -> g_static_h below
+//   h   [T*K, I] bf16   SwiGLU outputs, one row per routed pair    -> g_static_scratch
+//   y   [T*K, H] fp32   weighted expert outputs before the combine -> g_static_scratch
 //   flag                error bits                                 -> the caller's pointer
 // Nothing in the scratch has to start at zero: the gate/up kernel writes every h row the
-// down kernel reads, and the flag is overwritten by each call.  The array keeps the rows of
+// down kernel reads, the down kernel every y row the combine reads, and the flag is
+// overwritten by each call.  The array keeps the rows of
 // the last call after it ends.  There is ONE array per device, shared by every call on that
 // device: calls on one stream are ordered and safe; calls that can overlap (different
 // streams or host threads on the same device) race on it.
@@ -21,18 +23,18 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int64_t kStaticHElems = NVFP4_STATIC_MAX_H_ELEMS;   // 2^18 bf16 = 512 KB
+constexpr int64_t kStaticBytes = NVFP4_STATIC_SCRATCH_BYTES;   // 4 MiB
 constexpr int kMaxDevices = 64;
 
-__device__ __align__(256) __nv_bfloat16 g_static_h[kStaticHElems];
+__device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
 
 std::mutex g_lookup_mu;
-void *g_static_h_addr[kMaxDevices] = {};
+void *g_static_addr[kMaxDevices] = {};
 
-// Device address of g_static_h on the current device, looked up once per device.  The
-// lookup may load this library's device code, which is why the first call on a device
+// Device address of g_static_scratch on the current device, looked up once per device.
+// The lookup may load this library's device code, which is why the first call on a device
 // has to come before any stream capture on it begins.
-int static_scratch(__nv_bfloat16 **h) {
+int static_scratch(unsigned char **base) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -41,18 +43,21 @@ int static_scratch(__nv_bfloat16 **h) {
   }
   if (dev < 0 || dev >= kMaxDevices) return NVFP4_EINVAL;
   std::lock_guard<std::mutex> lock(g_lookup_mu);
-  if (!g_static_h_addr[dev]) {
+  if (!g_static_addr[dev]) {
     void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_h);
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess || !p) {
       set_last_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
       return NVFP4_ECUDA;
     }
-    g_static_h_addr[dev] = p;
+    g_static_addr[dev] = p;
   }
-  *h = static_cast<__nv_bfloat16 *>(g_static_h_addr[dev]);
+  *base = static_cast<unsigned char *>(g_static_addr[dev]);
   return NVFP4_OK;
 }
+
+// Bytes of h (rounded up to 256) and the offset of y inside the scratch.
+int64_t static_h_bytes(int64_t pairs, int64_t I) { return (pairs * I * 2 + 255) & ~int64_t(255); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -77,11 +82,12 @@ extern "C" int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *t
       !aligned16(s_gu) || !aligned16(s_dn) ||
       (reinterpret_cast<uintptr_t>(error_flag) & 3))
     return NVFP4_EINVAL;
-  // the fixed scratch bounds the batch: T*K*I bf16 values of h
-  if (T * K > kStaticHElems / I || !gemv_supported(T, H, I, K)) return NVFP4_ESHAPE;
+  // the fixed scratch bounds the batch: h (T*K*I bf16) and y (T*K*H fp32)
+  if (!gemv_supported(T, H, I, K)) return NVFP4_ESHAPE;
+  if (static_h_bytes(T * K, I) + T * K * H * 4 > kStaticBytes) return NVFP4_ESHAPE;
 
-  __nv_bfloat16 *h = nullptr;
-  if (int s = static_scratch(&h)) return s;
+  unsigned char *base = nullptr;
+  if (int s = static_scratch(&base)) return s;
 
   MoeArgs a = {};
   a.x = x;
@@ -100,7 +106,9 @@ extern "C" int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *t
   a.E = E;
   a.K = K;
   a.flag = error_flag;   // may be NULL: the kernels then skip the flag writes
-  a.h = h;
+  a.h = reinterpret_cast<__nv_bfloat16 *>(base);
+  a.y = reinterpret_cast<float *>(base + static_h_bytes(T * K, I));
   if (int s = launch_gemv_gateup(a, stream)) return s;
-  return launch_gemv_down(a, stream);
+  if (int s = launch_gemv_down(a, stream)) return s;
+  return gemv_fused_combine(T) ? NVFP4_OK : launch_combine_pairs(a, stream);
 }

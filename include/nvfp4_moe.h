@@ -178,9 +178,10 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
 
 /* ---------------------------------------------------------------- fixed-scratch forward */
 
-/* Largest T*K*I that moe_nvfp4_forward_static takes: its scratch holds T*K rows of I bf16
- * values (2^18 values = 512 KB; at I = 2048 and K = 8 that is T <= 16). */
-#define NVFP4_STATIC_MAX_H_ELEMS 262144
+/* Bytes of the fixed scratch of moe_nvfp4_forward_static: it holds T*K rows of I bf16 values
+ * (rounded up to 256 bytes) and T*K rows of H fp32 values, so a call needs
+ * roundup256(2*T*K*I) + 4*T*K*H <= 4 MiB (at H = 6144, I = 2048, K = 8: T <= 18). */
+#define NVFP4_STATIC_SCRATCH_BYTES 4194304
 
 /* The small-batch forward of moe_nvfp4_forward (its GEMV path: same kernels, same result)
  * without a caller workspace.  The pages have no counterpart to this call: it exists for
@@ -191,7 +192,7 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
  *   error_flag  [1] int32, may be NULL: receives what the workspace flag of
  *               moe_nvfp4_forward would (0, bit 0 = an id outside [0, E), bit 1 = a
  *               device-side wait gave up); overwritten by every call; 4-byte aligned.
- * Scratch: one array of NVFP4_STATIC_MAX_H_ELEMS bf16 per device, inside the library; no
+ * Scratch: one array of NVFP4_STATIC_SCRATCH_BYTES per device, inside the library; no
  * call allocates or frees memory.  Nothing in it needs to start at zero.  It keeps the last
  * call's intermediate values after that call ends.  All calls on a device share it, so
  * calls that can overlap in time (different streams, or different host threads, on the
@@ -199,8 +200,8 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
  * device looks the array's address up (cudaGetSymbolAddress): make that first call before
  * any stream capture begins on that device.
  * Errors: EINVAL (null or misaligned pointer, dimension <= 0), ESHAPE (the limits of
- * moe_nvfp4_forward, T*K*I > NVFP4_STATIC_MAX_H_ELEMS, or a shape the GEMV path does not
- * take: T*K > 1024, H > 6144 or I > 3072), ECUDA. */
+ * moe_nvfp4_forward, a batch whose h and y do not fit NVFP4_STATIC_SCRATCH_BYTES, or a
+ * shape the GEMV path does not take: T*K > 1024, H > 6144 or I > 6144), ECUDA. */
 NVFP4_API int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *topk_ids,
                                        const float *topk_w, int64_t T, int64_t H, int64_t I,
                                        int64_t E, int64_t K, const uint8_t *w_gu,

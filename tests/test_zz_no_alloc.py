@@ -74,9 +74,16 @@ def test_bad_id_sets_flag(nv):
 
 
 def test_batch_above_the_fixed_scratch_is_rejected(nv):
-    E, H, I, K = 16, 128, 2048, 8
-    T = 17                                   # 17 * 8 * 2048 > 2^18 bf16 values
-    layer = _layer(nv, E, H, I, seed=5)
-    x, ids, w = _batch(T, E, K, H, seed=6)
+    # per pair the scratch holds 2*I + 4*H bytes: 19 tokens x 8 pairs do not fit in 4 MiB
+    E, H, I, K, T = 1, 6144, 2048, 8, 19
+    dev = "cuda"
+    w_gu = torch.zeros((E, 2 * I, H // 2), dtype=torch.uint8, device=dev)
+    s_gu = torch.zeros((E, 2 * I, H // 16), dtype=torch.uint8, device=dev)
+    w_dn = torch.zeros((E, H, I // 2), dtype=torch.uint8, device=dev)
+    s_dn = torch.zeros((E, H, I // 16), dtype=torch.uint8, device=dev)
+    g = torch.ones((E,), dtype=torch.float32, device=dev)
+    x = torch.zeros((T, H), dtype=torch.bfloat16, device=dev)
+    ids = torch.zeros((T, K), dtype=torch.int32, device=dev)
+    w = torch.zeros((T, K), dtype=torch.float32, device=dev)
     with pytest.raises(nv.NVFP4Error, match="ESHAPE"):
-        nv.moe_nvfp4_forward_static(x, ids, w, *layer)
+        nv.moe_nvfp4_forward_static(x, ids, w, w_gu, s_gu, g, w_dn, s_dn, g)
