@@ -7,41 +7,60 @@
 //   code_i = E2M1(x_i / (dec(s) * g)), nearest even, saturating, sign kept; 0 if the
 //   divisor is 0.
 // Every step is the IEEE fp32 operation written (no reciprocal, no contraction), so the
-// bits are reproducible.  All three kernels stream HBM with 16-byte accesses.
-#include "common.cuh"
+// bits are reproducible.  The kernels stream HBM with 16-byte accesses.
+#include "pipeline.cuh"
 
 namespace nvfp4 {
 
-// ------------------------------------------------------------------ amax
-// Per-tensor max |x| as fp32 bits, merged with atomicMax (non-negative floats order like
-// their bit patterns).  grid = (blocks per tensor, n_tensors).
-__global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16 *__restrict__ x,
-                                                   int64_t per_tensor,
-                                                   uint32_t *__restrict__ amax_bits) {
-  const int t = blockIdx.y;
-  const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)t * per_tensor);
-  const int64_t nvec = per_tensor / 8;
-  uint32_t m = 0;  // max of |bf16| bit patterns (sign cleared) -- same order as values
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    uint4 v = ldg_stream(src + i);
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      m = max(m, w[j] & 0x7FFFu);
-      m = max(m, (w[j] >> 16) & 0x7FFFu);
-    }
+// ------------------------------------------------------------------ quantize
+// The element codes without a division.  With q = RN(|x| / d) (IEEE division) the E2M1 code
+// counts the rounding thresholds q passes: q > 0.25, q >= 0.75, q > 1.25, q >= 1.75, q > 2.5,
+// q >= 3.5, q > 5 (a midpoint goes to the even code).  Each threshold m has an even fp32
+// significand, so  RN(a) > m  <=>  a > m + u/2  and  RN(a) >= m  <=>  a >= m - u'/2, with u
+// and u' the fp32 spacings just above and just below m.  For an fp32 |x| and a real bound t,
+// |x| > t <=> |x| > RD32(t) and |x| >= t <=> |x| >= RU32(t), and RD32((m + u/2) d) is one
+// fused multiply-add rounded down, fma_rd(m, d, (u/2) d), because (u/2) d is a power-of-two
+// scaling of d and so exact.  The seven fp32 thresholds of a block therefore give the same
+// codes as dividing every element by d.  (For d below 2^-100 the scaled term could lose bits
+// to underflow, and the bounds are formed in fp64 instead, where the products are exact.)
+struct Thresholds {
+  float t[7];   // t[0], t[2], t[4], t[6]: compare with >; t[1], t[3], t[5]: with >=
+};
+
+__device__ __forceinline__ Thresholds block_thresholds(float d) {
+  Thresholds r;
+  if (d >= 0x1p-100f) {
+    r.t[0] = __fmaf_rd(0.25f, d, __fmul_rn(d, 0x1p-26f));
+    r.t[1] = __fmaf_ru(0.75f, d, -__fmul_rn(d, 0x1p-25f));
+    r.t[2] = __fmaf_rd(1.25f, d, __fmul_rn(d, 0x1p-24f));
+    r.t[3] = __fmaf_ru(1.75f, d, -__fmul_rn(d, 0x1p-24f));
+    r.t[4] = __fmaf_rd(2.5f, d, __fmul_rn(d, 0x1p-23f));
+    r.t[5] = __fmaf_ru(3.5f, d, -__fmul_rn(d, 0x1p-23f));
+    r.t[6] = __fmaf_rd(5.0f, d, __fmul_rn(d, 0x1p-22f));
+  } else {
+    const double dd = (double)d;
+    r.t[0] = __double2float_rd((0.25 + 0x1p-26) * dd);
+    r.t[1] = __double2float_ru((0.75 - 0x1p-25) * dd);
+    r.t[2] = __double2float_rd((1.25 + 0x1p-24) * dd);
+    r.t[3] = __double2float_ru((1.75 - 0x1p-24) * dd);
+    r.t[4] = __double2float_rd((2.5 + 0x1p-23) * dd);
+    r.t[5] = __double2float_ru((3.5 - 0x1p-23) * dd);
+    r.t[6] = __double2float_rd((5.0 + 0x1p-22) * dd);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  __shared__ uint32_t red[8];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = max(m, red[w]);
-    // bf16 bits << 16 are the fp32 bits of the same value
-    atomicMax(amax_bits + t, m << 16);
-  }
+  return r;
+}
+
+// E2M1 code of x for a block with divisor d > 0 (thresholds from block_thresholds(d)):
+// binary search over the seven thresholds, sign bit copied from x.
+__device__ __forceinline__ uint32_t e2m1_code(float x, const Thresholds &T) {
+  const float a = fabsf(x);
+  const bool b2 = a >= T.t[3];                         // code >= 4
+  const float t1 = b2 ? T.t[5] : T.t[1];               // code >= 6 / code >= 2
+  const bool b1 = a >= t1;
+  const float lo = b1 ? T.t[2] : T.t[0], hi = b1 ? T.t[6] : T.t[4];
+  const float t0 = b2 ? hi : lo;                       // the strict threshold above
+  const uint32_t c = (b2 ? 4u : 0u) + (b1 ? 2u : 0u) + (a > t0 ? 1u : 0u);
+  return c | ((__float_as_uint(x) >> 28) & 0x8u);
 }
 
 // g = amax / 2688, IEEE division, 1 for an all-zero tensor.
@@ -50,46 +69,190 @@ __device__ __forceinline__ float global_scale_from_amax(uint32_t amax_bits) {
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
-// ------------------------------------------------------------------ quantize
-// One thread per 8 elements (half a block); lanes 2i and 2i+1 share a block.
+// Workspace of nvfp4_quantize: [0] error flag, [4..4+n) amax bits, [4+n..4+2n) number of
+// CTAs whose amax share of tensor t is merged.
+constexpr int kQwsHeader = 4;
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait (one thread) until *p >= want; a wait that gives up sets bit 1 of ws[0].
+__device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t want, uint32_t *ws,
+                                           volatile int *abort) {
+  if (*abort) return false;
+  if (ld_acquire_gpu(p) >= want) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_gpu(p) < want) {
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(ws, (uint32_t)kFlagWaitTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// Quantize n tensors with one cooperative launch.  Warps 0-1 of every CTA take the amax of
+// tensor p over the CTA's share while warps 2-7 quantize the CTA's share of tensor p - 1,
+// which may start once every CTA has merged its amax of that tensor.  The amax warps wait
+// for their own CTA's quantize warps to finish tensor p - 2 before reading tensor p, so at
+// most about three tensors are in flight: a gate/up tensor of the layer is 50 MB, and the
+// quantize pass finds it in L2 right after the amax pass brought it in.  Each input byte
+// crosses HBM once.
+constexpr int kAmaxWarps = 2;
+constexpr int kAmaxThreads = 32 * kAmaxWarps;
+constexpr int kQuantThreads = 256 - kAmaxThreads;
+constexpr int kAmaxLoads = 16;   // 16-byte loads in flight per amax thread
+
+// One half block (8 elements) -> packed word; the block's scale code in *sc_out.  Lanes
+// 2i and 2i+1 hold the two halves of a block.
+__device__ __forceinline__ uint32_t quantize_half_block(uint4 v, float g, uint32_t *sc_out) {
+  const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                      bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+  float am = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) am = fmaxf(am, fabsf(f[k]));
+  am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+  const float sv = __fdiv_rn(__fdiv_rn(am, 6.0f), g);
+  const uint32_t sc = f32_to_e4m3(sv);
+  const float d = __fmul_rn(e4m3_to_f32(sc), g);
+  uint32_t word = 0;
+  if (d != 0.0f) {
+    const Thresholds T = block_thresholds(d);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) word |= e2m1_code(f[k], T) << (4 * k);
+  }
+  *sc_out = sc;
+  return word;
+}
+
+// L2 eviction-priority policies for the two reads of a tensor: the amax pass marks lines to
+// be kept (the quantize pass comes back for them), the quantize pass marks them as last use.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint4 ld_l2_hint(const void *ptr, uint64_t policy) {
+  uint4 r;
+  asm volatile("ld.global.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(ptr), "l"(policy));
+  return r;
+}
+
 __global__ void __launch_bounds__(256) quantize_kernel(
-    const __nv_bfloat16 *__restrict__ x, int64_t per_tensor, int64_t n_half_blocks,
-    const uint32_t *__restrict__ amax_bits, uint8_t *__restrict__ packed,
-    uint8_t *__restrict__ scales, float *__restrict__ global_scale) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int lane = threadIdx.x & 31;
-  // Warp-uniform loop so the pair shuffle always runs with all 32 lanes; lanes past the
-  // end compute on zeros and store nothing.  n_half_blocks is even, so both lanes of a
-  // pair are in range together.
-  for (int64_t hb0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-       hb0 < n_half_blocks; hb0 += stride) {
-    const int64_t hb = hb0 + lane;
-    const bool active = hb < n_half_blocks;
-    const int64_t e0 = (active ? hb : hb0) * 8;   // first element
-    const int t = (int)(e0 / per_tensor);           // tensor index
-    const float g = global_scale_from_amax(__ldg(amax_bits + t));
-    if (active && e0 == (int64_t)t * per_tensor) global_scale[t] = g;
+    const __nv_bfloat16 *__restrict__ x, int64_t per_tensor, int n_tensors,
+    uint32_t *__restrict__ ws, uint8_t *__restrict__ packed, uint8_t *__restrict__ scales,
+    float *__restrict__ global_scale) {
+  __shared__ int s_abort;
+  __shared__ int s_qdone;          // tensors this CTA has quantized
+  __shared__ uint32_t s_red[kAmaxWarps];
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    s_qdone = 0;
+  }
+  __syncthreads();
+  volatile int *abort = &s_abort;
+  uint32_t *amax_bits = ws + kQwsHeader;
+  uint32_t *merged = amax_bits + n_tensors;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nvec = per_tensor / 8;                    // 16-byte vectors = half blocks
+  const int64_t v0 = nvec * blockIdx.x / gridDim.x, v1 = nvec * (blockIdx.x + 1) / gridDim.x;
 
-    uint4 v = active ? ldg_stream(x + e0) : make_uint4(0, 0, 0, 0);
-    float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-    float amax = 0.0f;
+  if (warp < kAmaxWarps) {
+    const uint64_t keep = l2_policy_evict_last();
+    for (int p = 0; p < n_tensors; ++p) {
+      if (threadIdx.x == 0 && p >= 2) {   // keep the tensors in flight few
+        const uint64_t t0 = global_timer_ns();
+        while (*(volatile int *)&s_qdone < p - 1 && !*abort) {
+          if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(ws, (uint32_t)kFlagWaitTimeout);
+            *abort = 1;
+          }
+        }
+      }
+      named_sync(1, kAmaxThreads);
+      const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)p * per_tensor);
+      uint32_t m = 0;   // max of |bf16| bit patterns (same order as the values)
+      int64_t i = v0 + threadIdx.x;
+      for (; i + (kAmaxLoads - 1) * kAmaxThreads < v1; i += kAmaxLoads * kAmaxThreads) {
+        uint4 v[kAmaxLoads];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        for (int k = 0; k < kAmaxLoads; ++k) v[k] = ld_l2_hint(src + i + k * kAmaxThreads, keep);
+#pragma unroll
+        for (int k = 0; k < kAmaxLoads; ++k) {
+          const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+        }
+      }
+      for (; i < v1; i += kAmaxThreads) {
+        const uint4 v = ld_l2_hint(src + i, keep);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (lane == 0) s_red[warp] = m;
+      named_sync(1, kAmaxThreads);
+      if (threadIdx.x == 0) {
+        for (int w = 1; w < kAmaxWarps; ++w) m = max(m, s_red[w]);
+        if (m) atomicMax(amax_bits + p, m << 16);   // bf16 bits << 16 = fp32 bits
+        __threadfence();
+        atomicAdd(merged + p, 1u);
+      }
+    }
+    return;
+  }
 
-    const float s = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
-    const uint32_t sc = f32_to_e4m3(s);
-    const float d = __fmul_rn(e4m3_to_f32(sc), g);
-    uint32_t word = 0;
-    if (d != 0.0f) {
+  // ---- quantize: one thread per half block, four half blocks per thread per pass
+  const uint64_t last_use = l2_policy_evict_first();
+  const int qt = threadIdx.x - kAmaxThreads;
+  // the share boundaries are made even, so both halves of a block fall in one share
+  const int64_t q0 = v0 & ~int64_t(1);
+  const int64_t q1 = blockIdx.x + 1 == gridDim.x ? nvec : (v1 & ~int64_t(1));
+  for (int t = 0; t < n_tensors; ++t) {
+    if (qt == 0) wait_count(merged + t, gridDim.x, ws, abort);
+    named_sync(2, kQuantThreads);
+    const float g = global_scale_from_amax(__ldcg(amax_bits + t));
+    if (blockIdx.x == 0 && qt == 0) global_scale[t] = g;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)t * per_tensor);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(packed) + (int64_t)t * nvec;
+    uint8_t *sdst = scales + (int64_t)t * (nvec / 2);
+    // warp-uniform loop (the pair shuffle needs all lanes)
+    for (int64_t i0 = q0 + (qt & ~31); i0 < q1; i0 += 4 * kQuantThreads) {
+      uint4 v[4];
+      bool act[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= f32_to_e2m1(__fdiv_rn(f[i], d)) << (4 * i);
+      for (int k = 0; k < 4; ++k) {
+        const int64_t i = i0 + k * kQuantThreads + lane;
+        act[k] = i < q1;
+        v[k] = act[k] ? ld_l2_hint(src + i, last_use) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t sc;
+        const uint32_t word = quantize_half_block(v[k], g, &sc);
+        const int64_t i = i0 + k * kQuantThreads + lane;
+        if (act[k]) {
+          dst[i] = word;
+          if ((i & 1) == 0) sdst[i >> 1] = (uint8_t)sc;
+        }
+      }
     }
-    if (active) {
-      reinterpret_cast<uint32_t *>(packed)[hb] = word;
-      if ((hb & 1) == 0) scales[hb >> 1] = (uint8_t)sc;
-    }
+    named_sync(2, kQuantThreads);
+    if (qt == 0) *(volatile int *)&s_qdone = t + 1;
   }
 }
 
@@ -155,7 +318,7 @@ using namespace nvfp4;
 
 extern "C" size_t nvfp4_quantize_workspace_size(int64_t n_tensors, int64_t, int64_t) {
   if (n_tensors <= 0) return 0;
-  return (size_t)ceil_div(n_tensors * 4, 256) * 256;
+  return (size_t)ceil_div((kQwsHeader + 2 * n_tensors) * 4, 256) * 256;
 }
 
 extern "C" int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t rows,
@@ -165,6 +328,7 @@ extern "C" int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t
   if (!x || !packed || !scales || !global_scale || n_tensors <= 0 || rows <= 0 || cols <= 0)
     return NVFP4_EINVAL;
   if (cols % 32 != 0) return NVFP4_ESHAPE;
+  if (n_tensors >= (int64_t(1) << 24)) return NVFP4_ESHAPE;
   // 16-byte loads of x, 4-byte stores of packed codes
   if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(packed) & 3) ||
       (reinterpret_cast<uintptr_t>(global_scale) & 3))
@@ -173,22 +337,39 @@ extern "C" int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t
       (reinterpret_cast<uintptr_t>(workspace) & 3))
     return NVFP4_EWORKSPACE;
   const int64_t per = rows * cols;
-  uint32_t *amax = static_cast<uint32_t *>(workspace);
-  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t) * n_tensors, stream);
+  uint32_t *ws = static_cast<uint32_t *>(workspace);
+  cudaError_t e =
+      cudaMemsetAsync(ws, 0, sizeof(uint32_t) * (kQwsHeader + 2 * n_tensors), stream);
   if (e != cudaSuccess) {
     set_last_cuda_error(e);
     return NVFP4_ECUDA;
   }
-  // blocks per tensor: enough to fill the GPU a few times over in total
-  int64_t bpt = ceil_div(per / 8, 256 * 8);
-  int64_t want = ceil_div((int64_t)kNumSMs * 8, n_tensors);
-  if (bpt > want) bpt = want;
-  if (bpt < 1) bpt = 1;
-  amax_kernel<<<dim3((unsigned)bpt, (unsigned)n_tensors), 256, 0, stream>>>(x, per, amax);
-  if (int s = check_launch()) return s;
-  const int64_t n_hb = n_tensors * per / 8;
-  quantize_kernel<<<grid_for(n_hb, 256), 256, 0, stream>>>(x, per, n_hb, amax, packed, scales,
-                                                            global_scale);
+  // a cooperative launch: every CTA is resident, so no CTA waits on one that has not started
+  int dev = 0, sms = kNumSMs, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel, 256, 0);
+  if (e != cudaSuccess || per_sm <= 0) {
+    set_last_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
+    return NVFP4_ECUDA;
+  }
+  const int ctas = sms * (per_sm < 4 ? per_sm : 4);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, quantize_kernel, x, per, (int)n_tensors, ws, packed, scales,
+                         global_scale);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return NVFP4_ECUDA;
+  }
   return check_launch();
 }
 

@@ -60,7 +60,10 @@ NVFP4_API const char *nvfp4_last_cuda_error(void);
 
 /* ---------------------------------------------------------------- codec */
 
-/* Bytes of workspace nvfp4_quantize needs (a per-tensor amax accumulator). */
+/* Bytes of workspace nvfp4_quantize needs: an error word, a per-tensor amax accumulator and
+ * a per-tensor count of merged amax shares.  After the call, the first int32 of the workspace is 0, or
+ * has bit 1 set if a device-side wait gave up (the outputs are then invalid); it can be read
+ * with moe_nvfp4_read_error_flag. */
 NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t n_tensors, int64_t rows, int64_t cols);
 
 /* Quantize n_tensors bf16 tensors of shape [rows, cols] to NVFP4 (page "GLM-5-NVFP4-MTP",
@@ -73,6 +76,8 @@ NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t n_tensors, int64_t rows, 
  * d = decoded s * g; code_i = E2M1(x_i / d) (nearest, ties to even, saturating at 6, sign
  * kept, so a small negative value gives 0x8); all codes 0 when d == 0.  Every step is an
  * IEEE fp32 operation rounded to nearest even, so results are reproducible bit for bit.
+ * One cooperative kernel reads each tensor from HBM once: the quantize pass of a tensor
+ * follows its amax pass while the tensor is still in L2. 
  * Requires cols % 32 == 0.  NaN/Inf inputs give unspecified codes.
  * Alignment: x 16 bytes, packed and global_scale 4 bytes, workspace 4 bytes.
  * Errors: EINVAL (null pointer, dimension <= 0, misaligned pointer), ESHAPE (cols % 32 != 0),
