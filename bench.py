@@ -47,6 +47,16 @@ DOWN_BYTES_PER_EXPERT = H * (I // 2 + I // 16)            # 7,077,888
 EXPERT_BYTES = GATEUP_BYTES_PER_EXPERT + DOWN_BYTES_PER_EXPERT
 
 
+def measured_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary (profiles/), or None
+    when no capture of the current kernel is recorded."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            return json.load(f).get(kernel, {}).get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -264,12 +274,14 @@ def run_ours(args, rank, world, device):
     tokens_total = T * K_steps * world
     value = tokens_total / (ms_total / 1e3)
 
-    if T <= 64:   # HBM-bound: the gate/up GEMV streams 2/3 of the expert bytes
+    gemv = path == 1 or (path == 0 and T <= 64)
+    if gemv:   # HBM-bound: the gate/up GEMV streams 2/3 of the expert bytes
         gu_ms = stages["gate_up"]
         achieved = uniq * GATEUP_BYTES_PER_EXPERT / (gu_ms / 1e3) / 1e9
-        roof = {"kernel": "gemv_gateup_kernel (gate/up GEMV + SwiGLU)", "bound": "hbm",
+        kname = "gemv_gateup_kernel" if T == 1 else "gemv_mma_kernel<0>"
+        roof = {"kernel": kname + " (gate/up + SwiGLU)", "bound": "hbm",
                 "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(kname),
                 "algorithmic_bytes": uniq * GATEUP_BYTES_PER_EXPERT,
                 "peak_source": peaks["source"] + " (burst copy)"}
     else:
@@ -288,11 +300,13 @@ def run_ours(args, rank, world, device):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": K_steps, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 weights; f16/bf16 products, f32 accumulation",
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) bf16 weights quantized to NVFP4)",
         "config": {"workload": wl.name if E == 256 else wl.name.replace("E=256", f"E={E}"),
                    "T": T, "H": H, "I": I, "E": E, "K": K,
-                   "weights": "NVFP4 (E2M1 + E4M3 per 16 + fp32 per tensor), 5.4 GB resident",
+                   "weights": "NVFP4 (E2M1 + E4M3 per 16 + fp32 per tensor), "
+                              f"{E * EXPERT_BYTES / 1e9:.2f} GB resident",
                    "l2": "inputs larger than L2: every step routes new tokens over 5.4 GB of "
                          "expert weights (>126 MB L2)",
                    "timing": f"CUDA graph of {G} steps replayed, CUDA events",
@@ -304,7 +318,8 @@ def run_ours(args, rank, world, device):
         "stages_ms": stages, "marked_step_ms": marked_step,
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": (2 if (path == 1 or (path == 0 and T <= 64)) else 4) * K_steps,
+        # GEMV: gate/up + down (+ combine for T > 1); GEMM: route, gather, 2 GEMMs, combine
+        "gpu_launches": ((2 if T == 1 else 3) if gemv else 5) * K_steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -384,12 +399,19 @@ def run_codec(args, nv, rank, world, device, peaks):
         ms = e0.elapsed_time(e1) / args.steps
         gbs = elts * 2.5625 / (ms / 1e3) / 1e9
         res[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]}
-    return {"metric": "NVFP4 codec GB/s (whole layer)", "value": res["quantize"]["GB/s"],
+    qa = res["quantize"]["GB/s"]
+    roof = {"kernel": "quantize_kernel (amax + quantize, one cooperative launch)",
+            "bound": "hbm", "achieved": qa, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": qa / peaks["hbm_gbs"], "traffic": None,
+            "algorithmic_bytes": elts * 2.5625, "peak_source": peaks["source"] + " (burst copy)"}
+    return {"metric": "NVFP4 codec GB/s (whole layer)", "value": qa,
             "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": res["quantize"]["ms"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "elements": elts},
-            "codec": res, "gpu_launches": 2 * 2 * args.steps}
+            "config": {"workload": wl.name, "elements": elts,
+                       "l2": "inputs (19.3 GB bf16) larger than L2"},
+            "roofline": roof, "codec": res,
+            "gpu_launches": 2 * args.steps}   # one quantize launch per projection per step
 
 
 # ----------------------------------------------------------------------------- reference arm
