@@ -462,10 +462,11 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- plumbing
-def barrier(world):
+def barrier(world, device=None):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if device is None or torch.device(device).type == "cuda":
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(v, world, device):
