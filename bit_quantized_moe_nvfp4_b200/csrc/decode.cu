@@ -294,7 +294,7 @@ __device__ __forceinline__ void to_f16x32(const uint4 (&v)[4], float s, uint32_t
 constexpr int kRedSlots = 4;
 
 struct Smem {
-  uint32_t bars, stages, red, smax, ids, act_e, act_off, misc, slot, run, hist, yk, total;
+  uint32_t bars, stages, red, smax, ids, act_e, act_off, misc, slot, run, hist, yk, hpre, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -303,7 +303,7 @@ __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v
 __host__ __device__ inline int red_slot_floats(int cw, int red_vals) { return cw * red_vals + 8; }
 
 __host__ __device__ inline Smem smem_layout(int S, uint32_t stage_bytes, int cw, int red_vals,
-                                            int n, int E, int yk_floats) {
+                                            int n, int E, int yk_floats, uint32_t hpre_bytes = 0) {
   Smem s;
   uint32_t o = 0;
   s.bars = o;
@@ -314,7 +314,7 @@ __host__ __device__ inline Smem smem_layout(int S, uint32_t stage_bytes, int cw,
   s.red = o;
   o += 4 * kRedSlots * red_slot_floats(cw, red_vals);
   s.smax = o;
-  o += 4 * cw * 4;
+  o += 4 * (cw * 8 + 8);
   s.ids = o;
   o += 4 * n;
   const int na = min(E, n);
@@ -333,6 +333,9 @@ __host__ __device__ inline Smem smem_layout(int S, uint32_t stage_bytes, int cw,
   o = align_up(o, 16);
   s.yk = o;
   o += 4 * yk_floats;
+  o = align_up(o, 16);
+  s.hpre = o;
+  o += hpre_bytes;
   s.total = align_up(o, 128);
   return s;
 }
@@ -973,7 +976,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
   const int E = (int)a.E;
   constexpr int RV = RD * NT;
   const int RS = red_slot_floats(CW, RV);
-  const Smem L = smem_layout(S, stage_bytes, CW, RV, n, E, n * nb);
+  const Smem L = smem_layout(S, stage_bytes, CW, RV, n, E, n * nb,
+                             NT == 1 ? (uint32_t)(8 * I * 2) : 0u);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint64_t *empty = full + S;
   uint64_t *rfull = empty + S;
@@ -1085,6 +1089,57 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
     int pair_of[NT];
     int cur_a = -1, ngroups = 0, cnt = 0, slot0 = 0;
     int it = 0;
+    // One token: the h rows of all (at most 8) slots are scaled to f16 once, up front, into
+    // shared memory, so an expert switch costs no global load and no barrier.
+    constexpr int kPre = 8;
+    const int n_valid = R.act_off[n_act];
+    const bool pre = NT == 1 && n_valid <= kPre;
+    uint4 *hpre = reinterpret_cast<uint4 *>(smem + L.hpre);   // [kPre][I/8] f16
+    float *pspre = smax + CW * kPre;                          // [kPre]
+    if (NT == 1 && pre) {
+      float m[kPre];
+#pragma unroll
+      for (int sl = 0; sl < kPre; ++sl) {
+        float mm = 0.f;
+        if (owns && sl < n_valid) {
+          const uint4 *hp = reinterpret_cast<const uint4 *>(a.h + (int64_t)sl * I + chunk * 16);
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const uint4 v = __ldcg(hp + k2);
+            hpre[(size_t)sl * (I / 8) + chunk * 2 + k2] = v;   // raw bf16 for now
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mm = fmaxf(mm, fmaxf(fabsf(bf16_lo(w4[k])), fabsf(bf16_hi(w4[k]))));
+          }
+        }
+        m[sl] = warp_max(mm);
+      }
+      if (lane == 0)
+#pragma unroll
+        for (int sl = 0; sl < kPre; ++sl) smax[cw * kPre + sl] = m[sl];
+      named_sync(1, nthreads_c);
+#pragma unroll 1
+      for (int sl = 0; sl < n_valid; ++sl) {
+        float mm = 0.f;
+        for (int w = 0; w < CW; ++w) mm = fmaxf(mm, smax[w * kPre + sl]);
+        const int p = prescale_exponent(mm);
+        if (cw == 0 && lane == 0) pspre[sl] = exp2i(-p);
+        const float sp = exp2i(p);
+        if (owns) {
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            uint4 &v = hpre[(size_t)sl * (I / 8) + chunk * 2 + k2];
+            const uint4 r = v;
+            v = make_uint4(f16x2_rn(bf16_lo(r.x) * sp, bf16_hi(r.x) * sp),
+                           f16x2_rn(bf16_lo(r.y) * sp, bf16_hi(r.y) * sp),
+                           f16x2_rn(bf16_lo(r.z) * sp, bf16_hi(r.z) * sp),
+                           f16x2_rn(bf16_lo(r.w) * sp, bf16_hi(r.w) * sp));
+          }
+        }
+      }
+      named_sync(1, nthreads_c);
+    }
     for (int s = 0; s < n_stages; ++s) {
       const int ai = s / chunks_per_expert;
       const int r0 = n0 + (s % chunks_per_expert) * RD;
@@ -1102,7 +1157,22 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
       for (int grp = 0; grp < ngroups; ++grp, ++it) {
         const int nt = min(NT, cnt - grp * NT);
         const bool last = grp == ngroups - 1;
-        if (ngroups > 1 || new_expert) {
+        if (NT == 1 && pre && (ngroups > 1 || new_expert)) {
+          const int pr = pairs_of_expert<NT>(R.ids, n, R.act_e[ai], grp * NT, lane);
+          pair_of[0] = __shfl_sync(0xFFFFFFFFu, pr, 0);
+          const int slot = slot0 + grp;
+          pscale[0] = pspre[slot];
+          if (owns) {
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const uint4 v = hpre[(size_t)slot * (I / 8) + chunk * 2 + k2];
+              xh[0][4 * k2] = v.x;
+              xh[0][4 * k2 + 1] = v.y;
+              xh[0][4 * k2 + 2] = v.z;
+              xh[0][4 * k2 + 3] = v.w;
+            }
+          }
+        } else if (ngroups > 1 || new_expert) {
           // h rows of this group's slots (slot = slot0 + grp*NT + i), scaled to f16
           const int pr = pairs_of_expert<NT>(R.ids, n, R.act_e[ai], grp * NT, lane);
           const uint4 *hp[NT];
@@ -1267,7 +1337,8 @@ int launch_down_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
   ctas = max64(ctas, ceil_div(a.H, max_nb));
   const int nb = (int)ceil_div(a.H, ctas);
   ctas = ceil_div(a.H, nb);
-  const Smem L = smem_layout(S, stage_bytes, CW, RD * NT, n, (int)a.E, n * nb);
+  const uint32_t hpre = NT == 1 ? (uint32_t)(8 * a.I * 2) : 0u;   // one token: h preloaded
+  const Smem L = smem_layout(S, stage_bytes, CW, RD * NT, n, (int)a.E, n * nb, hpre);
   const int fit = resident_blocks(gemv_down_kernel<NT, RD, S>, 32 * (CW + 2), L.total);
   if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
   return launch_pdl(gemv_down_kernel<NT, RD, S>, dim3((unsigned)ctas), dim3(32 * (CW + 2)),
