@@ -24,6 +24,9 @@
 // rounded to f16.  bf16 has 8 significant bits and f16 11, so this is exact for every
 // element above 2^-31 * max|x_t| (smaller ones lose bits below f16's subnormal grid); the
 // dot products are rescaled by 2^-p_t in fp32.
+#include <mutex>
+#include <vector>
+
 #include "moe.cuh"
 #include "pipeline.cuh"
 
@@ -1278,8 +1281,27 @@ int num_sms() {
 }
 
 // Blocks of kernel k that fit on one SM at once with this block size and shared memory.
+// Blocks of kernel k that fit on one SM at once with this block size and shared memory.  The
+// answer (and the shared-memory attribute it needs) is cached per kernel, device and size, so
+// a steady stream of calls pays for the query once.
 template <typename Kern>
 int resident_blocks(Kern k, int threads, size_t smem) {
+  struct Entry {
+    const void *fn;
+    int dev, threads;
+    size_t smem;
+    int nb;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const void *fn = reinterpret_cast<const void *>(k);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry &c : cache)
+      if (c.fn == fn && c.dev == dev && c.threads == threads && c.smem == smem) return c.nb;
+  }
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
     set_last_cuda_error(e);
@@ -1291,6 +1313,8 @@ int resident_blocks(Kern k, int threads, size_t smem) {
     set_last_cuda_error(e);
     return -1;
   }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() < 256) cache.push_back({fn, dev, threads, smem, nb});
   return nb;
 }
 

@@ -21,9 +21,10 @@
  *     a failed launch; nvfp4_last_cuda_error() then names the CUDA error.
  *   - Layouts are row-major.  A packed row stores element 2j in the LOW nibble of byte j and
  *     element 2j+1 in the HIGH nibble.  Block scales run along the contiguous dimension.
- *   - The library keeps no global state apart from a per-thread copy of the last CUDA error
- *     and the fixed array of moe_nvfp4_forward_static; calls on different streams may run
- *     concurrently if their workspaces differ.
+ *   - The library keeps no global state apart from a per-thread copy of the last CUDA error,
+ *     the fixed array of moe_nvfp4_forward_static and a cache of per-kernel launch
+ *     attributes (occupancy); calls on different streams may run concurrently if their
+ *     workspaces differ.
  */
 #ifndef NVFP4_MOE_H
 #define NVFP4_MOE_H
