@@ -628,7 +628,9 @@ constexpr int kGuRedFloats = kGuWarps * 16 * kGuTok + 2 * kGuTok;   // per reduc
 __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1,
                                               uint32_t a2, uint32_t a3, uint32_t b0,
                                               uint32_t b1) {
-  asm volatile(
+  // not volatile: the MMA has no effect besides its outputs, so the compiler may schedule
+  // the decode of the next operands around it
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
