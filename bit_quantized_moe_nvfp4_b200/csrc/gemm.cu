@@ -125,6 +125,20 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams &p, int tile, int
 
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
 
+// v[i] for a runtime i < N without dynamic register indexing.
+template <int N>
+__device__ __forceinline__ float pick(const float (&v)[N], int i) {
+  float r = v[0];
+#pragma unroll
+  for (int k = 1; k < N; ++k)
+    if (i == k) r = v[k];
+  return r;
+}
+
+// silu(z) = z / (1 + e^-z) with the fast exponential and division (a few ulp of fp32; h is
+// rounded to bf16 right after).  For z below about -88, e^-z is infinite and the quotient 0.
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
 // ------------------------------------------------------------------ dequantize
 // NW packed words (8 E2M1 codes each) with their NW/2 block scales (one byte per 16
 // elements, low bytes first) -> 4*NW packed 16-bit pairs, each the exact product e2m1*e4m3:
@@ -397,25 +411,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float g = __ldg(p.gscale + t.e);
       const int ncols = round16(t.nvalid);
+      // per-column factors of the tile (slot c0 + lane of each 32-column chunk), all loaded
+      // before the first accumulator read: 2^-p (gate/up) or the routing weight (down)
+      constexpr int kChunks = (BN + 31) / 32;
+      float colf[kChunks];
+      {
+        int pr[kChunks];
+#pragma unroll
+        for (int ch = 0; ch < kChunks; ++ch) {
+          const int col = 32 * ch + lane;
+          pr[ch] = (col < t.nvalid && p.mode == 1) ? __ldg(a.perm + t.slot0 + col) : 0;
+        }
+#pragma unroll
+        for (int ch = 0; ch < kChunks; ++ch) {
+          const int col = 32 * ch + lane;
+          colf[ch] = col >= t.nvalid ? 0.f
+                     : (p.mode == 0 ? a.xscale[t.slot0 + col] : __ldg(a.w + pr[ch])) * g;
+        }
+      }
       for (int c0 = 0; ok && c0 < ncols; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c0, v);
+        const float cf = pick<kChunks>(colf, c0 >> 5);
         if (p.mode == 0) {
           const int64_t j = (int64_t)t.mt * 64 + (m >> 1);
-          const float xl = (c0 + lane < t.nvalid) ? a.xscale[t.slot0 + c0 + lane] * g : 0.f;
+          const float xl = cf;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float val = __uint_as_float(v[c]) * __shfl_sync(0xFFFFFFFFu, xl, c);
             const float other = __shfl_xor_sync(0xFFFFFFFFu, val, 1);
             if (!(lane & 1) && c0 + c < t.nvalid) {
-              const float hv = silu_f32(val) * other;       // val = gate, other = up
+              const float hv = silu_fast(val) * other;      // val = gate, other = up
               a.h[(int64_t)(t.slot0 + c0 + c) * I + j] = __float2bfloat16_rn(hv);
             }
           }
         } else {
           const int64_t n = (int64_t)t.mt * BM + m;
-          const int sl = t.slot0 + c0 + lane;
-          const float wl = (c0 + lane < t.nvalid) ? __ldg(a.w + a.perm[sl]) * g : 0.f;
+          const float wl = cf;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float wc = __shfl_sync(0xFFFFFFFFu, wl, c);
