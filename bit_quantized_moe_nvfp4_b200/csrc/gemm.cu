@@ -81,7 +81,11 @@ constexpr uint32_t kPBytes = BM * BK / 2;     // packed weights (4 or 8 KB)
 constexpr int kSB = BK / 16;                  // block-scale bytes per row per stage
 constexpr uint32_t kSmemB = 0;
 constexpr uint32_t kSmemP = kSmemB + kS * kBBytes;
-constexpr uint32_t kSmemBars = kSmemP + kS * kPBytes;
+// epilogue staging: two buffers of one 32-column chunk of the output tile (down: 32 slots x
+// 128 rows fp32 = 16 KB; gate/up: 32 slots x 64 bf16 = 4 KB), written to HBM by TMA stores
+constexpr uint32_t kOutBufBytes = 32 * BM * 4;
+constexpr uint32_t kSmemOut = kSmemP + kS * kPBytes;
+constexpr uint32_t kSmemBars = kSmemOut + 2 * kOutBufBytes;
 constexpr uint32_t kSmemMisc = kSmemBars + 8 * (2 * kS + 2 * kSA + 4);
 constexpr uint32_t kSmemTotal = kSmemMisc + 16 + 1024;   // + alignment slack
 static_assert(kSmemTotal <= 227 * 1024, "shared memory budget");
@@ -189,7 +193,8 @@ __device__ __forceinline__ void dequant_words(const uint32_t (&words)[NW], uint3
 // ------------------------------------------------------------------ the GEMM kernel
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                const __grid_constant__ CUtensorMap tmap_b, GemmParams p) {
+                const __grid_constant__ CUtensorMap tmap_b,
+                const __grid_constant__ CUtensorMap tmap_out, GemmParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem =
       smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);   // 1024-byte aligned
@@ -404,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                 // epilogue warps are consecutive)
     const int m = q * 32 + lane;                // accumulator row (TMEM lane)
     int tc = 0;
+    int nchunk_out = 0;                         // chunks sent through the staging buffers
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tc) {
       const TileInfo t = tile_info(p, tile, n_act);
       const int acc = tc & 1;
@@ -433,33 +439,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c0, v);
         const float cf = pick<kChunks>(colf, c0 >> 5);
+        // A chunk whose 32 slots all belong to the tile goes out through shared memory and
+        // one TMA store; a partial chunk (the expert's last few slots) is stored directly,
+        // so no row of the next expert is touched.
+        const bool full_chunk = c0 + 32 <= t.nvalid;
+        unsigned char *ob = smem + kSmemOut + (size_t)(nchunk_out & 1) * kOutBufBytes;
+        if (full_chunk) {
+          // the store that last read this buffer (two chunks ago) is done: see below
+          named_sync(3, 128);
+        }
         if (p.mode == 0) {
-          const int64_t j = (int64_t)t.mt * 64 + (m >> 1);
-          const float xl = cf;
+          const int jl = q * 16 + (lane >> 1);     // column of h within the m tile (0..63)
+          const int64_t j = (int64_t)t.mt * 64 + jl;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float val = __uint_as_float(v[c]) * __shfl_sync(0xFFFFFFFFu, xl, c);
+            const float val = __uint_as_float(v[c]) * __shfl_sync(0xFFFFFFFFu, cf, c);
             const float other = __shfl_xor_sync(0xFFFFFFFFu, val, 1);
-            if (!(lane & 1) && c0 + c < t.nvalid) {
-              const float hv = silu_fast(val) * other;      // val = gate, other = up
-              a.h[(int64_t)(t.slot0 + c0 + c) * I + j] = __float2bfloat16_rn(hv);
+            const __nv_bfloat16 hv = __float2bfloat16_rn(silu_fast(val) * other);  // gate, up
+            if (!(lane & 1)) {
+              if (full_chunk)
+                reinterpret_cast<__nv_bfloat16 *>(ob)[c * 64 + jl] = hv;
+              else if (c0 + c < t.nvalid)
+                a.h[(int64_t)(t.slot0 + c0 + c) * I + j] = hv;
             }
           }
         } else {
           const int64_t n = (int64_t)t.mt * BM + m;
-          const float wl = cf;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float wc = __shfl_sync(0xFFFFFFFFu, wl, c);
-            if (n < H && c0 + c < t.nvalid)
-              a.y[(int64_t)(t.slot0 + c0 + c) * H + n] = __uint_as_float(v[c]) * wc;
+            const float yv = __uint_as_float(v[c]) * __shfl_sync(0xFFFFFFFFu, cf, c);
+            if (full_chunk)
+              reinterpret_cast<float *>(ob)[c * BM + m] = yv;
+            else if (n < H && c0 + c < t.nvalid)
+              a.y[(int64_t)(t.slot0 + c0 + c) * H + n] = yv;
           }
+        }
+        if (full_chunk) {
+          fence_proxy_async_smem();   // generic writes -> visible to the TMA engine
+          named_sync(3, 128);
+          if (warp == kWarpEpi && lane == 0) {
+            if (p.mode == 0)
+              tma_store_2d(&tmap_out, t.mt * 64, t.slot0 + c0, ob);
+            else
+              tma_store_2d(&tmap_out, t.mt * BM, t.slot0 + c0, ob);
+            bulk_commit_group();
+            bulk_wait_group_read<1>();   // the other buffer may be rewritten
+          }
+          ++nchunk_out;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[acc]);
     }
+    if (warp == kWarpEpi && lane == 0) bulk_wait_group_all();   // every TMA store is done
   }
 
   // all roles are done: release tensor memory
@@ -571,6 +604,18 @@ int launch_gemm(const MoeArgs &a, int mode, cudaStream_t s) {
                2, mode == 0 ? (const void *)a.xs : (const void *)a.h,
                (uint64_t)p.K, brows, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return NVFP4_ECUDA;
+  // outputs for the epilogue's TMA stores: h [T*K + pad, I] bf16 in boxes of 32 slots x 64,
+  // or y [T*K, H] fp32 in boxes of 32 slots x 128
+  CUtensorMap to;
+  if (mode == 0) {
+    if (make_map(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h, (uint64_t)a.I, brows, 64, 32,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+      return NVFP4_ECUDA;
+  } else {
+    if (make_map(&to, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.y, (uint64_t)a.H,
+                 (uint64_t)(a.T * a.K), BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return NVFP4_ECUDA;
+  }
   cudaError_t e =
       cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTotal);
   if (e != cudaSuccess) {
@@ -580,7 +625,7 @@ int launch_gemm(const MoeArgs &a, int mode, cudaStream_t s) {
   int dev = 0, sms = kNumSMs;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return launch_pdl(gemm_kernel, dim3(sms), dim3(kThreads), kSmemTotal, s, tw, tb, p);
+  return launch_pdl(gemm_kernel, dim3(sms), dim3(kThreads), kSmemTotal, s, tw, tb, to, p);
 }
 
 }  // namespace
