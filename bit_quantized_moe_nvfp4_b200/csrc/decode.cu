@@ -39,13 +39,13 @@ namespace {
 #define NVFP4_GEMV_STAGES 2
 #endif
 #ifndef NVFP4_GEMV_PAIRS
-#define NVFP4_GEMV_PAIRS 4
+#define NVFP4_GEMV_PAIRS 8
 #endif
 #ifndef NVFP4_GEMV_DOWN_ROWS
 #define NVFP4_GEMV_DOWN_ROWS 32
 #endif
 #ifndef NVFP4_GEMV_CTAS_PER_SM
-#define NVFP4_GEMV_CTAS_PER_SM 3
+#define NVFP4_GEMV_CTAS_PER_SM 2
 #endif
 #ifndef NVFP4_GEMV_DOWN_STAGES
 #define NVFP4_GEMV_DOWN_STAGES NVFP4_GEMV_STAGES
@@ -363,7 +363,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *a
 // finalizes.  Each computing lane owns 32 consecutive elements (16 packed bytes, 2 block
 // scales) of every row; a stage holds P gate rows and the P matching up rows of one expert.
 template <int NT, int P, int S>
-__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 3 : 1)
+__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
     gemv_gateup_kernel(MoeArgs a, uint32_t stage_bytes) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_abort;
