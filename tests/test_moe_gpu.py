@@ -77,6 +77,30 @@ def test_edge_cases(nv, path):
     assert nv.moe_nvfp4_read_error_flag(ws) == 0
 
 
+@pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
+def test_single_token_edge_cases(nv, path):
+    """One token (the single-token GEMV kernels): an expert picked three times, another
+    twice, an out-of-range id, a reduction length that is not a multiple of 128; then a
+    token whose ids are all out of range (zero output)."""
+    E, H, I, K = 8, 192, 128, 8
+    layer = Layer(E, H, I, seed=9)
+    x = synth.activations_bf16(1, H, 9)
+    ids = torch.tensor([[3, 3, 1, E, 3, 0, 7, 1]], dtype=torch.int32)
+    w = torch.arange(1, K + 1, dtype=torch.float32).view(1, K) / 36.0
+    ws = nv.alloc_moe_workspace(1, H, I, E, K)
+    out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *layer.dev, workspace=ws,
+                               path=path)
+    assert nv.moe_nvfp4_read_error_flag(ws) & 1
+    ref, ref64, bad = layer.oracle_forward(x, ids, w)
+    assert bad == 1
+    compare_moe(out, ref, ref64)
+    bad_ids = torch.full((1, K), -1, dtype=torch.int32)
+    out = nv.moe_nvfp4_forward(x.cuda(), bad_ids.cuda(), w.cuda(), *layer.dev, workspace=ws,
+                               path=path)
+    assert nv.moe_nvfp4_read_error_flag(ws) & 1
+    assert torch.all(out == 0)
+
+
 # ----------------------------------------------------------------------------- full size
 class FullLayer:
     """All 256 experts of the H=6144, I=2048 layer on the GPU, quantized by the GPU
