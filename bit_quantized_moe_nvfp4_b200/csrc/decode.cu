@@ -50,6 +50,9 @@ namespace {
 #ifndef NVFP4_GEMV_DOWN_STAGES
 #define NVFP4_GEMV_DOWN_STAGES NVFP4_GEMV_STAGES
 #endif
+#ifndef NVFP4_GEMV_DOWN_WARPS
+#define NVFP4_GEMV_DOWN_WARPS 4
+#endif
 #ifndef NVFP4_GEMV_DOWN_CTAS_PER_SM
 #define NVFP4_GEMV_DOWN_CTAS_PER_SM 2
 #endif
@@ -57,6 +60,7 @@ constexpr int kStages = NVFP4_GEMV_STAGES;       // shared-memory ring depth
 constexpr int kPairs = NVFP4_GEMV_PAIRS;         // gate/up row pairs per stage
 constexpr int kDownRows = NVFP4_GEMV_DOWN_ROWS;  // rows per stage (down kernel)
 constexpr int kDownStages = NVFP4_GEMV_DOWN_STAGES;
+constexpr int kDownWarps = NVFP4_GEMV_DOWN_WARPS;   // compute warps (down kernel)
 constexpr int kMaxConsumerWarps = 6;
 constexpr int64_t kGemvMaxPairs = 1024;  // T*K handled by the GEMV path
 
@@ -564,13 +568,14 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
         }
         named_sync(1, nthreads_c);   // smax is rewritten by the next load
       }
-      // partial dot products of all 2P rows (rows past np hold stale data and are ignored)
+      // partial dot products of the 2*np loaded rows (the others stay zero and are ignored)
       float flat[RV];
 #pragma unroll
       for (int v = 0; v < RV; ++v) flat[v] = 0.f;
       if (owns && have) {
 #pragma unroll
         for (int r = 0; r < 2 * P; ++r) {
+          if (r % P >= np) continue;   // warp-uniform: a short stage skips its stale rows
           const uint4 q = *reinterpret_cast<const uint4 *>(st + (size_t)r * rowb + chunk * 16);
           const unsigned char *sp = (r < P) ? spg : spu;
           const uint32_t sc2 = *reinterpret_cast<const unsigned short *>(
@@ -964,38 +969,38 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
   }
 }
 
-// ================================================================== down + combine
-// CTA c owns output rows [n0, n0 + nb) for every active expert.  Warp 0 produces, warps
-// 1..CW compute with lanes owning 16 consecutive elements (8 packed bytes, 1 block scale),
-// warp CW+1 finalizes.  Per-pair results stay in shared memory (yk) and are combined in
-// ascending k at the end.
-template <int NT, int RD, int S>
-__global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
+// ================================================================== down + combine (one token)
+// CTA c owns output rows [n0, n0 + nb) (nb <= kDownRows) for every active expert; a stage is
+// one expert's nb rows.  Warp 0 produces; warps 1..CW compute, each taking whole rows (row r
+// of a stage belongs to warp r % CW), with lane l owning the 16-byte units l, l + 32, ... of
+// the packed row (32 elements, two blocks, each), so a row's dot product needs only the
+// warp's own shuffle reduction.  The h rows of all slots arrive in shared memory with one
+// bulk copy and are scaled to f16 once.  The per-pair results stay in shared memory (yk)
+// and are combined in ascending k at the end.
+template <int UPL, int CW, int S>
+__global__ void __launch_bounds__(32 * (CW + 1))
     gemv_down_kernel(MoeArgs a, uint32_t stage_bytes, int nb) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_abort;
-  const int CW = blockDim.x / 32 - 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t H = a.H, I = a.I, K = a.K, T = a.T;
-  const int n = (int)(T * K);
+  const int64_t H = a.H, I = a.I, K = a.K;
+  const int n = (int)K;   // one token: pair k is slot-routed directly
   const int E = (int)a.E;
-  constexpr int RV = RD * NT;
-  const int RS = red_slot_floats(CW, RV);
-  const Smem L = smem_layout(S, stage_bytes, CW, RV, n, E, n * nb,
-                             NT == 1 ? (uint32_t)(8 * I * 2) : 0u);
+  constexpr int RPW = (kDownRows + CW - 1) / CW;   // rows of a stage per warp
+  static_assert((RPW & (RPW - 1)) == 0 && RPW <= 32, "rows per warp must be a power of two");
+  const Smem L = smem_layout(S, stage_bytes, CW, 0, n, E, n * nb, (uint32_t)(n * I * 2));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint64_t *empty = full + S;
-  uint64_t *rfull = empty + S;
-  uint64_t *rfree = rfull + kRedSlots;
+  uint64_t *hbar = empty + S;
   unsigned char *stage_base = smem + L.stages;
-  float *red = reinterpret_cast<float *>(smem + L.red);
-  float *smax = reinterpret_cast<float *>(smem + L.smax);
+  float *pss = reinterpret_cast<float *>(smem + L.smax);   // [n] 2^-p of each slot
   CtaRoute R{reinterpret_cast<int *>(smem + L.ids), reinterpret_cast<int *>(smem + L.act_e),
              reinterpret_cast<int *>(smem + L.act_off), reinterpret_cast<int *>(smem + L.misc)};
   int *hist = reinterpret_cast<int *>(smem + L.hist);
   int *slot_of = reinterpret_cast<int *>(smem + L.slot);
   int *run = reinterpret_cast<int *>(smem + L.run);
   float *yk = reinterpret_cast<float *>(smem + L.yk);
+  uint4 *hsm = reinterpret_cast<uint4 *>(smem + L.hpre);   // [n][I/8]: bf16, then scaled f16
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -1003,10 +1008,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], CW);
     }
-    for (int s = 0; s < kRedSlots; ++s) {
-      mbar_init(&rfull[s], CW);
-      mbar_init(&rfree[s], 1);
-    }
+    mbar_init(hbar, 1);
     mbar_init_fence();
   }
   // The ids were complete before the gate/up kernel let this grid start; reading them
@@ -1018,19 +1020,16 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
 
   const int n0 = blockIdx.x * nb;
   const int n1 = min((int)H, n0 + nb);
+  const int nr = max(0, n1 - n0);   // rows of every stage
   const uint32_t rowb = (uint32_t)(I / 2), sclb = (uint32_t)(I / 16);
-  const int rows_per_expert = n1 > n0 ? (n1 - n0) : 0;
-  const int chunks_per_expert = (rows_per_expert + RD - 1) / RD;
-  const int n_stages = n_act * chunks_per_expert;
+  const uint32_t srows = (uint32_t)nb;   // row capacity of a stage
+  const int n_stages = nr > 0 ? n_act : 0;
 
   if (warp == 0) {
     if (lane == 0) {
       int s = 0;
       for (; s < n_stages; ++s) {
-        const int ai = s / chunks_per_expert;
-        const int r0 = n0 + (s % chunks_per_expert) * RD;
-        const int nr = min(RD, n1 - r0);
-        const int e = R.act_e[ai];
+        const int e = R.act_e[s];
         const int idx = s % S;
         if (s >= S && (*(volatile int *)&s_abort || !mbar_wait(&empty[idx], ((s / S) - 1) & 1))) {
           if (!*(volatile int *)&s_abort) report_timeout(a.flag);
@@ -1038,12 +1037,12 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
           break;
         }
         unsigned char *st = stage_base + (size_t)idx * stage_bytes;
-        const int64_t row = (int64_t)e * H + r0;
-        const int64_t ls = (int64_t)r0 * sclb;
+        const int64_t row = (int64_t)e * H + n0;
+        const int64_t ls = (int64_t)n0 * sclb;
         const uint32_t span = (uint32_t)(((ls + nr * sclb + 15) & ~15ll) - (ls & ~15ll));
         mbar_arrive_expect_tx(&full[idx], (uint32_t)nr * rowb + span);
         bulk_g2s(st, a.w_dn + row * rowb, nr * rowb, &full[idx]);
-        bulk_g2s_span(st + RD * rowb, a.s_dn + (int64_t)e * H * sclb, ls, nr * sclb, &full[idx]);
+        bulk_g2s_span(st + srows * rowb, a.s_dn + (int64_t)e * H * sclb, ls, nr * sclb, &full[idx]);
       }
       const int issued = s;
       for (int t = max(0, issued - S); t < issued; ++t)
@@ -1052,221 +1051,137 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2))
     return;
   }
 
-  const int nthreads_cf = (CW + 1) * 32;   // compute + finalizer threads (combine)
-  if (warp == CW + 1) {
-    // ------------------------------------------------ finalizer
-    int it = 0;
-    for (int s = 0; s < n_stages; ++s) {
-      const int ai = s / chunks_per_expert;
-      const int r0 = n0 + (s % chunks_per_expert) * RD;
-      const int nr = min(RD, n1 - r0);
-      const int slot0 = R.act_off[ai];
-      const int cnt = R.act_off[ai + 1] - slot0;
-      const float g = __ldg(a.g_dn + R.act_e[ai]);
-      for (int grp = 0; grp * NT < cnt; ++grp, ++it) {
-        const int nt = min(NT, cnt - grp * NT);
-        const int sl = it % kRedSlots;
-        const bool ok = warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag);
-        const float *rb = red + (size_t)sl * RS;
-        if (ok && lane < nr * nt) {
-          const int rr = lane / nt, i = lane % nt;
-          float sum = 0.f;
-          for (int w = 0; w < CW; ++w) sum += rb[w * RV + rr * NT + i];
-          const float ps = rb[CW * RV + i];
-          const int pair = __float_as_int(rb[CW * RV + 4 + i]);
-          const int slot = slot0 + grp * NT + i;
-          yk[(size_t)slot * nb + (r0 - n0) + rr] = sum * g * ps * __ldg(a.w + pair);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&rfree[sl]);
+  // ------------------------------------------------ compute warps
+  const int cw = warp - 1;
+  const int nthreads_c = CW * 32;
+  pdl_wait();   // h is written by the gate/up kernel
+  pdl_launch_dependents();
+  const int n_valid = R.act_off[n_act];   // slots 0..n_valid-1 are the rows of h in use
+  if (cw == 0 && lane == 0 && n_valid > 0) {
+    const uint32_t bytes = (uint32_t)((int64_t)n_valid * I * 2);
+    mbar_arrive_expect_tx(hbar, bytes);
+    bulk_g2s(hsm, a.h, bytes, hbar);
+  }
+  if (n_valid > 0) warp_wait(hbar, 0, &s_abort, a.flag);
+  // Scale each slot by an exact power of two into f16 (warp cw takes slots cw, cw + CW, ...),
+  // stored unit-transposed: 16-byte piece i of unit u (32 elements) goes to index i * U + u, so
+  // the per-stage reloads below read consecutive 16-byte pieces across the lanes.
+  const int U = (int)(I / 32);   // 16-byte units per packed row = 64-byte units per h row
+  for (int sl = cw; sl < n_valid; sl += CW) {
+    uint4 *row = hsm + (size_t)sl * (4 * U);
+    uint4 v[UPL][4];
+    float mm = 0.f;
+#pragma unroll
+    for (int k = 0; k < UPL; ++k) {
+      const int u = lane + 32 * k;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[k][i] = u < U ? row[4 * u + i] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w4[4] = {v[k][i].x, v[k][i].y, v[k][i].z, v[k][i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mm = fmaxf(mm, fmaxf(fabsf(bf16_lo(w4[j])), fabsf(bf16_hi(w4[j]))));
       }
     }
-  } else {
-    // ------------------------------------------------ compute warps
-    pdl_wait();   // h is written by the gate/up kernel
-    pdl_launch_dependents();
-    const int cw = warp - 1;
-    const int nthreads_c = CW * 32;
-    const int chunk = cw * 32 + lane;              // 16-element chunk owned by this lane
-    const bool owns = chunk < (int)(I / 16);
-    uint32_t xh[NT][8];
-    float pscale[NT];
-    int pair_of[NT];
-    int cur_a = -1, ngroups = 0, cnt = 0, slot0 = 0;
-    int it = 0;
-    // One token: the h rows of all (at most 8) slots are scaled to f16 once, up front, into
-    // shared memory, so an expert switch costs no global load and no barrier.
-    constexpr int kPre = 8;
-    const int n_valid = R.act_off[n_act];
-    const bool pre = NT == 1 && n_valid <= kPre;
-    uint4 *hpre = reinterpret_cast<uint4 *>(smem + L.hpre);   // [kPre][I/8] f16
-    float *pspre = smax + CW * kPre;                          // [kPre]
-    if (NT == 1 && pre) {
-      float m[kPre];
+    mm = warp_max(mm);   // also orders every lane's reads before the writes below
+    const int p = prescale_exponent(mm);
+    const float sp = exp2i(p);
 #pragma unroll
-      for (int sl = 0; sl < kPre; ++sl) {
-        float mm = 0.f;
-        if (owns && sl < n_valid) {
-          const uint4 *hp = reinterpret_cast<const uint4 *>(a.h + (int64_t)sl * I + chunk * 16);
+    for (int k = 0; k < UPL; ++k) {
+      const int u = lane + 32 * k;
+      if (u < U) {
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const uint4 v = __ldcg(hp + k2);
-            hpre[(size_t)sl * (I / 8) + chunk * 2 + k2] = v;   // raw bf16 for now
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mm = fmaxf(mm, fmaxf(fabsf(bf16_lo(w4[k])), fabsf(bf16_hi(w4[k]))));
-          }
-        }
-        m[sl] = warp_max(mm);
-      }
-      if (lane == 0)
-#pragma unroll
-        for (int sl = 0; sl < kPre; ++sl) smax[cw * kPre + sl] = m[sl];
-      named_sync(1, nthreads_c);
-#pragma unroll 1
-      for (int sl = 0; sl < n_valid; ++sl) {
-        float mm = 0.f;
-        for (int w = 0; w < CW; ++w) mm = fmaxf(mm, smax[w * kPre + sl]);
-        const int p = prescale_exponent(mm);
-        if (cw == 0 && lane == 0) pspre[sl] = exp2i(-p);
-        const float sp = exp2i(p);
-        if (owns) {
-#pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            uint4 &v = hpre[(size_t)sl * (I / 8) + chunk * 2 + k2];
-            const uint4 r = v;
-            v = make_uint4(f16x2_rn(bf16_lo(r.x) * sp, bf16_hi(r.x) * sp),
-                           f16x2_rn(bf16_lo(r.y) * sp, bf16_hi(r.y) * sp),
-                           f16x2_rn(bf16_lo(r.z) * sp, bf16_hi(r.z) * sp),
-                           f16x2_rn(bf16_lo(r.w) * sp, bf16_hi(r.w) * sp));
-          }
+        for (int i = 0; i < 4; ++i) {
+          const uint4 q = v[k][i];
+          row[i * U + u] = make_uint4(f16x2_rn(bf16_lo(q.x) * sp, bf16_hi(q.x) * sp),
+                                      f16x2_rn(bf16_lo(q.y) * sp, bf16_hi(q.y) * sp),
+                                      f16x2_rn(bf16_lo(q.z) * sp, bf16_hi(q.z) * sp),
+                                      f16x2_rn(bf16_lo(q.w) * sp, bf16_hi(q.w) * sp));
         }
       }
-      named_sync(1, nthreads_c);
     }
-    for (int s = 0; s < n_stages; ++s) {
-      const int ai = s / chunks_per_expert;
-      const int r0 = n0 + (s % chunks_per_expert) * RD;
-      const int idx = s % S;
-      const bool new_expert = ai != cur_a;
-      if (new_expert) {
-        cur_a = ai;
-        slot0 = R.act_off[ai];
-        cnt = R.act_off[ai + 1] - slot0;
-        ngroups = (cnt + NT - 1) / NT;
+    if (lane == 0) pss[sl] = exp2i(-p);
+    __syncwarp();
+  }
+  named_sync(1, nthreads_c);
+
+  for (int s = 0; s < n_stages; ++s) {
+    const int idx = s % S;
+    const int slot0 = R.act_off[s];
+    const int cnt = R.act_off[s + 1] - slot0;   // > 1 only for a repeated expert id
+    const float g = __ldg(a.g_dn + R.act_e[s]);
+    const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
+    const unsigned char *st = stage_base + (size_t)idx * stage_bytes;
+    const unsigned char *sbase = st + srows * rowb + (((int64_t)n0 * sclb) & 15);
+    for (int c = 0; c < cnt; ++c) {
+      const int slot = slot0 + c;
+      uint32_t xh[UPL][16];
+      const uint4 *hrow = hsm + (size_t)slot * (4 * U);
+#pragma unroll
+      for (int k = 0; k < UPL; ++k) {
+        const int u = lane + 32 * k;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = u < U ? hrow[i * U + u] : make_uint4(0u, 0u, 0u, 0u);
+          xh[k][4 * i] = v.x;
+          xh[k][4 * i + 1] = v.y;
+          xh[k][4 * i + 2] = v.z;
+          xh[k][4 * i + 3] = v.w;
+        }
       }
-      const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
-      const unsigned char *st = stage_base + (size_t)idx * stage_bytes;
-      const unsigned char *sbase = st + RD * rowb + (((int64_t)r0 * sclb) & 15);
-      for (int grp = 0; grp < ngroups; ++grp, ++it) {
-        const int nt = min(NT, cnt - grp * NT);
-        const bool last = grp == ngroups - 1;
-        if (NT == 1 && pre && (ngroups > 1 || new_expert)) {
-          const int pr = pairs_of_expert<NT>(R.ids, n, R.act_e[ai], grp * NT, lane);
-          pair_of[0] = __shfl_sync(0xFFFFFFFFu, pr, 0);
-          const int slot = slot0 + grp;
-          pscale[0] = pspre[slot];
-          if (owns) {
+      float flat[RPW];
 #pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-              const uint4 v = hpre[(size_t)slot * (I / 8) + chunk * 2 + k2];
-              xh[0][4 * k2] = v.x;
-              xh[0][4 * k2 + 1] = v.y;
-              xh[0][4 * k2 + 2] = v.z;
-              xh[0][4 * k2 + 3] = v.w;
+      for (int i = 0; i < RPW; ++i) flat[i] = 0.f;
+      if (have) {
+        // two rows at a time (independent chains); a missing second row re-reads the first
+#pragma unroll
+        for (int i = 0; i < RPW; i += 2) {
+          const int ra = cw + i * CW;
+          if (ra >= nr) break;   // warp-uniform
+          const int rb = ra + CW < nr ? ra + CW : ra;
+          float acc_a = 0.f, acc_b = 0.f;
+#pragma unroll
+          for (int k = 0; k < UPL; ++k) {
+            const int u = lane + 32 * k;
+            if (u < U) {
+              const uint4 qa = *reinterpret_cast<const uint4 *>(st + (size_t)ra * rowb + 16 * u);
+              const uint4 qb = *reinterpret_cast<const uint4 *>(st + (size_t)rb * rowb + 16 * u);
+              const uint32_t sa = e4m3x2_to_f16x2(
+                  *reinterpret_cast<const unsigned short *>(sbase + (size_t)ra * sclb + 2 * u));
+              const uint32_t sb = e4m3x2_to_f16x2(
+                  *reinterpret_cast<const unsigned short *>(sbase + (size_t)rb * sclb + 2 * u));
+              const float a0 = dot16(qa.x, qa.y, &xh[k][0]);
+              const float b0 = dot16(qb.x, qb.y, &xh[k][0]);
+              const float a1 = dot16(qa.z, qa.w, &xh[k][8]);
+              const float b1 = dot16(qb.z, qb.w, &xh[k][8]);
+              acc_a = fmaf(a1, f16_hi(sa), fmaf(a0, f16_lo(sa), acc_a));
+              acc_b = fmaf(b1, f16_hi(sb), fmaf(b0, f16_lo(sb), acc_b));
             }
           }
-        } else if (ngroups > 1 || new_expert) {
-          // h rows of this group's slots (slot = slot0 + grp*NT + i), scaled to f16
-          const int pr = pairs_of_expert<NT>(R.ids, n, R.act_e[ai], grp * NT, lane);
-          const uint4 *hp[NT];
-          float m[NT];
-#pragma unroll
-          for (int i = 0; i < NT; ++i) {
-            pair_of[i] = __shfl_sync(0xFFFFFFFFu, pr, min(i, nt - 1));
-            const int slot = slot0 + grp * NT + min(i, nt - 1);
-            hp[i] = reinterpret_cast<const uint4 *>(a.h + (int64_t)slot * I + chunk * 16);
-            float mm = 0.f;
-            if (owns) {
-#pragma unroll
-              for (int k2 = 0; k2 < 2; ++k2) {
-                const uint4 v = __ldcg(hp[i] + k2);
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  mm = fmaxf(mm, fmaxf(fabsf(bf16_lo(w4[k])), fabsf(bf16_hi(w4[k]))));
-              }
-            }
-            m[i] = warp_max(mm);
-          }
-          if (lane == 0)
-#pragma unroll
-            for (int i = 0; i < NT; ++i) smax[cw * 4 + i] = m[i];
-          named_sync(1, nthreads_c);
-#pragma unroll
-          for (int i = 0; i < NT; ++i) {
-            float mm = 0.f;
-            for (int w = 0; w < CW; ++w) mm = fmaxf(mm, smax[w * 4 + i]);
-            const int p = prescale_exponent(mm);
-            pscale[i] = exp2i(-p);
-            if (owns) {
-              const float sp = exp2i(p);
-#pragma unroll
-              for (int k2 = 0; k2 < 2; ++k2) {
-                const uint4 v = __ldcg(hp[i] + k2);
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  xh[i][4 * k2 + k] = f16x2_rn(bf16_lo(w4[k]) * sp, bf16_hi(w4[k]) * sp);
-              }
-            }
-          }
-          named_sync(1, nthreads_c);
+          flat[i] = acc_a;
+          if (i + 1 < RPW) flat[i + 1] = acc_b;
         }
-        float flat[RV];
-#pragma unroll
-        for (int v = 0; v < RV; ++v) flat[v] = 0.f;
-        if (owns && have) {
-#pragma unroll
-          for (int r = 0; r < RD; ++r) {
-            const uint2 q = *reinterpret_cast<const uint2 *>(st + (size_t)r * rowb + chunk * 8);
-            const float sc = e4m3_to_f32(sbase[(size_t)r * sclb + chunk]);
-#pragma unroll
-            for (int i = 0; i < NT; ++i) flat[r * NT + i] = dot16(q.x, q.y, &xh[i][0]) * sc;
-          }
-        }
-        if (last) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[idx]);
-        }
-        const float tot = warp_reduce_many<RV>(flat, lane);
-        constexpr int SH = 5 - Log2<RV>::value;
-        const int sl = it % kRedSlots;
-        if (it >= kRedSlots) warp_wait(&rfree[sl], ((it / kRedSlots) - 1) & 1, &s_abort, a.flag);
-        float *rb = red + (size_t)sl * RS;
-        if ((lane & ((1 << SH) - 1)) == 0) rb[cw * RV + (lane >> SH)] = tot;
-        if (cw == 0 && lane < NT) {
-          rb[CW * RV + lane] = pick<NT>(pscale, lane);
-          rb[CW * RV + 4 + lane] = __int_as_float(pick<NT>(pair_of, lane));
-        }
+      }
+      if (c == cnt - 1) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(&rfull[sl]);
+        if (lane == 0) mbar_arrive(&empty[idx]);   // this warp is done reading the stage
       }
+      const float tot = warp_reduce_many<RPW>(flat, lane);
+      constexpr int SH = 5 - Log2<RPW>::value;
+      const int r = cw + (lane >> SH) * CW;
+      if ((lane & ((1 << SH) - 1)) == 0 && r < nr) yk[(size_t)slot * nb + r] = tot * g * pss[slot];
     }
   }
-  named_sync(2, nthreads_cf);   // every y of this CTA is in yk
-  // combine in ascending k: out[t, n] = sum_k y(slot(t, k))[n]
+  named_sync(2, nthreads_c);   // every y of this CTA is in yk
+  // combine in ascending k: out[n0 + o] = sum_k w[k] * y(slot(k))[o]
   const int ctid = threadIdx.x - 32;
-  const int nbr = n1 - n0;
-  for (int o = ctid; o < T * nbr; o += nthreads_cf) {
-    const int t = o / nbr, rr = o % nbr;
+  for (int o = ctid; o < nr; o += nthreads_c) {
     float acc = 0.f;
     for (int k = 0; k < K; ++k) {
-      const int sl = slot_of[t * K + k];
-      if (sl >= 0) acc += yk[(size_t)sl * nb + rr];
+      const int sl = slot_of[k];
+      if (sl >= 0) acc += yk[(size_t)sl * nb + o] * __ldg(a.w + k);
     }
-    a.out[(int64_t)t * H + n0 + rr] = __float2bfloat16_rn(acc);
+    a.out[n0 + o] = __float2bfloat16_rn(acc);
   }
 }
 
@@ -1352,22 +1267,19 @@ int launch_mma(const MoeArgs &a, cudaStream_t s) {
   return launch_mma_cfg<MODE, 2>(a, s);
 }
 
-template <int NT, int RD, int S>
+template <int UPL, int CW, int S>
 int launch_down_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
-  const int CW = (int)ceil_div(a.I, 512);
-  const uint32_t stage_bytes = (uint32_t)(RD * (a.I / 2) + span_bytes(RD * (a.I / 16)));
   const int n = (int)(a.T * a.K);
-  // enough CTAs for the GPU, and few enough rows per CTA that the per-pair results fit
-  int64_t ctas = (int64_t)num_sms() * ctas_per_sm;
-  const int64_t max_nb = max64(1, (32 * 1024) / (4 * (n > 1 ? n : 1)));
-  ctas = max64(ctas, ceil_div(a.H, max_nb));
-  const int nb = (int)ceil_div(a.H, ctas);
-  ctas = ceil_div(a.H, nb);
-  const uint32_t hpre = NT == 1 ? (uint32_t)(8 * a.I * 2) : 0u;   // one token: h preloaded
-  const Smem L = smem_layout(S, stage_bytes, CW, RD * NT, n, (int)a.E, n * nb, hpre);
-  const int fit = resident_blocks(gemv_down_kernel<NT, RD, S>, 32 * (CW + 2), L.total);
+  // enough CTAs for the GPU, and at most kDownRows rows per CTA (one stage per expert)
+  const int64_t want = max64((int64_t)num_sms() * ctas_per_sm, ceil_div(a.H, kDownRows));
+  const int nb = (int)ceil_div(a.H, want);
+  const int64_t ctas = ceil_div(a.H, nb);
+  const uint32_t stage_bytes =
+      align_up((uint32_t)(nb * (a.I / 2)) + span_bytes(nb * (a.I / 16)), 128);
+  const Smem L = smem_layout(S, stage_bytes, CW, 0, n, (int)a.E, n * nb, (uint32_t)(n * a.I * 2));
+  const int fit = resident_blocks(gemv_down_kernel<UPL, CW, S>, 32 * (CW + 1), L.total);
   if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
-  return launch_pdl(gemv_down_kernel<NT, RD, S>, dim3((unsigned)ctas), dim3(32 * (CW + 2)),
+  return launch_pdl(gemv_down_kernel<UPL, CW, S>, dim3((unsigned)ctas), dim3(32 * (CW + 1)),
                     L.total, s, a, stage_bytes, nb);
 }
 
@@ -1375,7 +1287,8 @@ int launch_down_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
 
 bool gemv_supported(int64_t T, int64_t H, int64_t I, int64_t K) {
   if (T * K > kGemvMaxPairs) return false;
-  if (T == 1)   // CUDA-core kernels: 32 (gate/up) or 16 (down) elements per lane, 6 warps
+  if (T == 1)   // CUDA-core kernels: gate/up lanes own 32 elements of a row (6 warps), down
+                // lanes up to three 32-element units
     return H <= 1024 * kMaxConsumerWarps && I <= 512 * kMaxConsumerWarps;
   const int64_t max_k = (int64_t)kGuWarps * kGuMaxChunks * 128;   // mma kernels
   return H <= max_k && I <= max_k;
@@ -1393,8 +1306,12 @@ int launch_gemv_gateup(const MoeArgs &a, cudaStream_t s) {
 }
 
 int launch_gemv_down(const MoeArgs &a, cudaStream_t s) {
-  if (gemv_fused_combine(a.T))
-    return launch_down_cfg<1, kDownRows, kDownStages>(a, s, NVFP4_GEMV_DOWN_CTAS_PER_SM);
+  if (gemv_fused_combine(a.T)) {   // one token: lanes own ceil(I / 1024) 16-byte units
+    const int c = NVFP4_GEMV_DOWN_CTAS_PER_SM;
+    if (a.I <= 1024) return launch_down_cfg<1, kDownWarps, kDownStages>(a, s, c);
+    if (a.I <= 2048) return launch_down_cfg<2, kDownWarps, kDownStages>(a, s, c);
+    return launch_down_cfg<3, kDownWarps, kDownStages>(a, s, c);
+  }
   return launch_mma<1>(a, s);
 }
 
