@@ -50,6 +50,9 @@ namespace {
 #ifndef NVFP4_GEMV_DOWN_STAGES
 #define NVFP4_GEMV_DOWN_STAGES NVFP4_GEMV_STAGES
 #endif
+#ifndef NVFP4_GEMV_DOWN_SPLIT
+#define NVFP4_GEMV_DOWN_SPLIT 1
+#endif
 #ifndef NVFP4_GEMV_DOWN_WARPS
 #define NVFP4_GEMV_DOWN_WARPS 4
 #endif
@@ -61,6 +64,7 @@ constexpr int kPairs = NVFP4_GEMV_PAIRS;         // gate/up row pairs per stage
 constexpr int kDownRows = NVFP4_GEMV_DOWN_ROWS;  // rows per stage (down kernel)
 constexpr int kDownStages = NVFP4_GEMV_DOWN_STAGES;
 constexpr int kDownWarps = NVFP4_GEMV_DOWN_WARPS;   // compute warps (down kernel)
+constexpr int kDownSplit = NVFP4_GEMV_DOWN_SPLIT;   // stages per expert (down kernel)
 constexpr int kMaxConsumerWarps = 6;
 constexpr int64_t kGemvMaxPairs = 1024;  // T*K handled by the GEMV path
 
@@ -403,6 +407,16 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
     mbar_init_fence();
   }
   pdl_wait();  // x and the ids come from earlier kernels
+  // One token: the compute lanes issue their activation loads first, so they are not
+  // queued behind the weight stream that starts once the routing is known.
+  const int chunk = (warp - 1) * 32 + lane;      // 32-element chunk owned by a compute lane
+  const bool owns = warp >= 1 && warp <= CW && chunk < (int)(H / 32);
+  uint4 xv[4];
+  if (NT == 1 && owns) {
+    const uint4 *xp = reinterpret_cast<const uint4 *>(a.x + chunk * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xv[i] = __ldcg(xp + i);
+  }
   const bool bad = cta_route(a.ids, n, E, R, hist);
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.flag) *a.flag = bad ? kFlagBadId : 0;
   pdl_launch_dependents();  // the down kernel may start routing and prefetching
@@ -493,8 +507,6 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
 
   // ------------------------------------------------ compute warps
   const int cw = warp - 1;                       // compute warp index
-  const int chunk = cw * 32 + lane;              // 32-element chunk owned by this lane
-  const bool owns = chunk < (int)(H / 32);
   const int nthreads_c = CW * 32;
   uint32_t xh[NT][16];
   float pscale[NT];                              // 2^-p per token of the current group
@@ -503,6 +515,30 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
   for (int i = 0; i < NT; ++i) loaded_tok[i] = -1;
   int cur_a = -1, ngroups = 0, cnt = 0;
   int s = 0, it = 0;
+  if (NT == 1 && U0 < U1) {
+    // One token: every pair is token 0, whose activations were loaded above; they are
+    // scaled to f16 before the first stage arrives.
+    float mx = 0.f;
+    if (owns) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t w4[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mx = fmaxf(mx, fmaxf(fabsf(bf16_lo(w4[k])), fabsf(bf16_hi(w4[k]))));
+      }
+    }
+    const float m = warp_max(mx);
+    if (lane == 0) smax[cw * 4] = m;
+    named_sync(1, nthreads_c);
+    float mm = 0.f;
+    for (int w = 0; w < CW; ++w) mm = fmaxf(mm, smax[w * 4]);
+    const int p = prescale_exponent(mm);
+    pscale[0] = exp2i(-p);
+    if (owns) to_f16x32(xv, exp2i(p), xh[0]);
+    loaded_tok[0] = 0;
+    named_sync(1, nthreads_c);   // smax is rewritten by any later load
+  }
   for (int64_t u = U0; u < U1; ++s) {
     const int ai = (int)(u / I);
     const int64_t j = u % I;
@@ -970,8 +1006,8 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
 }
 
 // ================================================================== down + combine (one token)
-// CTA c owns output rows [n0, n0 + nb) (nb <= kDownRows) for every active expert; a stage is
-// one expert's nb rows.  Warp 0 produces; warps 1..CW compute, each taking whole rows (row r
+// CTA c owns output rows [n0, n0 + nb) (nb <= kDownRows) for every active expert; a stage
+// holds srows of them (one expert's rows in ceil(nb / srows) stages).  Warp 0 produces; warps 1..CW compute, each taking whole rows (row r
 // of a stage belongs to warp r % CW), with lane l owning the 16-byte units l, l + 32, ... of
 // the packed row (32 elements, two blocks, each), so a row's dot product needs only the
 // warp's own shuffle reduction.  The h rows of all slots arrive in shared memory with one
@@ -979,7 +1015,7 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
 // and are combined in ascending k at the end.
 template <int UPL, int CW, int S>
 __global__ void __launch_bounds__(32 * (CW + 1))
-    gemv_down_kernel(MoeArgs a, uint32_t stage_bytes, int nb) {
+    gemv_down_kernel(MoeArgs a, uint32_t stage_bytes, int nb, int srows) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1020,16 +1056,18 @@ __global__ void __launch_bounds__(32 * (CW + 1))
 
   const int n0 = blockIdx.x * nb;
   const int n1 = min((int)H, n0 + nb);
-  const int nr = max(0, n1 - n0);   // rows of every stage
+  const int nr = max(0, n1 - n0);   // rows of this CTA (per expert)
   const uint32_t rowb = (uint32_t)(I / 2), sclb = (uint32_t)(I / 16);
-  const uint32_t srows = (uint32_t)nb;   // row capacity of a stage
-  const int n_stages = nr > 0 ? n_act : 0;
+  const int cpe = nr > 0 ? (nr + srows - 1) / srows : 0;   // stages per expert
+  const int n_stages = n_act * cpe;
 
   if (warp == 0) {
     if (lane == 0) {
       int s = 0;
       for (; s < n_stages; ++s) {
-        const int e = R.act_e[s];
+        const int e = R.act_e[s / cpe];
+        const int q0 = (s % cpe) * srows;           // first row of the stage (from n0)
+        const int nq = min(srows, nr - q0);
         const int idx = s % S;
         if (s >= S && (*(volatile int *)&s_abort || !mbar_wait(&empty[idx], ((s / S) - 1) & 1))) {
           if (!*(volatile int *)&s_abort) report_timeout(a.flag);
@@ -1037,12 +1075,12 @@ __global__ void __launch_bounds__(32 * (CW + 1))
           break;
         }
         unsigned char *st = stage_base + (size_t)idx * stage_bytes;
-        const int64_t row = (int64_t)e * H + n0;
-        const int64_t ls = (int64_t)n0 * sclb;
-        const uint32_t span = (uint32_t)(((ls + nr * sclb + 15) & ~15ll) - (ls & ~15ll));
-        mbar_arrive_expect_tx(&full[idx], (uint32_t)nr * rowb + span);
-        bulk_g2s(st, a.w_dn + row * rowb, nr * rowb, &full[idx]);
-        bulk_g2s_span(st + srows * rowb, a.s_dn + (int64_t)e * H * sclb, ls, nr * sclb, &full[idx]);
+        const int64_t row = (int64_t)e * H + n0 + q0;
+        const int64_t ls = (int64_t)(n0 + q0) * sclb;
+        const uint32_t span = (uint32_t)(((ls + nq * sclb + 15) & ~15ll) - (ls & ~15ll));
+        mbar_arrive_expect_tx(&full[idx], (uint32_t)nq * rowb + span);
+        bulk_g2s(st, a.w_dn + row * rowb, nq * rowb, &full[idx]);
+        bulk_g2s_span(st + srows * rowb, a.s_dn + (int64_t)e * H * sclb, ls, nq * sclb, &full[idx]);
       }
       const int issued = s;
       for (int t = max(0, issued - S); t < issued; ++t)
@@ -1065,39 +1103,34 @@ __global__ void __launch_bounds__(32 * (CW + 1))
   if (n_valid > 0) warp_wait(hbar, 0, &s_abort, a.flag);
   // Scale each slot by an exact power of two into f16 (warp cw takes slots cw, cw + CW, ...),
   // stored unit-transposed: 16-byte piece i of unit u (32 elements) goes to index i * U + u, so
-  // the per-stage reloads below read consecutive 16-byte pieces across the lanes.
+  // the per-stage reloads below read consecutive 16-byte pieces across the lanes.  Lane l
+  // reads pieces l, l + 32, ... (consecutive across the warp), and each group of 8 lanes
+  // writes 8 consecutive transposed pieces, so neither side has bank conflicts.
   const int U = (int)(I / 32);   // 16-byte units per packed row = 64-byte units per h row
   for (int sl = cw; sl < n_valid; sl += CW) {
     uint4 *row = hsm + (size_t)sl * (4 * U);
-    uint4 v[UPL][4];
+    uint4 v[4 * UPL];
     float mm = 0.f;
 #pragma unroll
-    for (int k = 0; k < UPL; ++k) {
-      const int u = lane + 32 * k;
+    for (int j = 0; j < 4 * UPL; ++j) {
+      const int pc = lane + 32 * j;   // piece in natural order: unit pc / 4, index pc % 4
+      v[j] = pc < 4 * U ? row[pc] : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[k][i] = u < U ? row[4 * u + i] : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t w4[4] = {v[k][i].x, v[k][i].y, v[k][i].z, v[k][i].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mm = fmaxf(mm, fmaxf(fabsf(bf16_lo(w4[j])), fabsf(bf16_hi(w4[j]))));
-      }
+      for (int k = 0; k < 4; ++k) mm = fmaxf(mm, fmaxf(fabsf(bf16_lo(w4[k])), fabsf(bf16_hi(w4[k]))));
     }
     mm = warp_max(mm);   // also orders every lane's reads before the writes below
     const int p = prescale_exponent(mm);
     const float sp = exp2i(p);
 #pragma unroll
-    for (int k = 0; k < UPL; ++k) {
-      const int u = lane + 32 * k;
-      if (u < U) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 q = v[k][i];
-          row[i * U + u] = make_uint4(f16x2_rn(bf16_lo(q.x) * sp, bf16_hi(q.x) * sp),
-                                      f16x2_rn(bf16_lo(q.y) * sp, bf16_hi(q.y) * sp),
-                                      f16x2_rn(bf16_lo(q.z) * sp, bf16_hi(q.z) * sp),
-                                      f16x2_rn(bf16_lo(q.w) * sp, bf16_hi(q.w) * sp));
-        }
+    for (int j = 0; j < 4 * UPL; ++j) {
+      const int pc = lane + 32 * j;
+      if (pc < 4 * U) {
+        const uint4 q = v[j];
+        row[(pc & 3) * U + (pc >> 2)] = make_uint4(f16x2_rn(bf16_lo(q.x) * sp, bf16_hi(q.x) * sp),
+                                                   f16x2_rn(bf16_lo(q.y) * sp, bf16_hi(q.y) * sp),
+                                                   f16x2_rn(bf16_lo(q.z) * sp, bf16_hi(q.z) * sp),
+                                                   f16x2_rn(bf16_lo(q.w) * sp, bf16_hi(q.w) * sp));
       }
     }
     if (lane == 0) pss[sl] = exp2i(-p);
@@ -1107,12 +1140,15 @@ __global__ void __launch_bounds__(32 * (CW + 1))
 
   for (int s = 0; s < n_stages; ++s) {
     const int idx = s % S;
-    const int slot0 = R.act_off[s];
-    const int cnt = R.act_off[s + 1] - slot0;   // > 1 only for a repeated expert id
-    const float g = __ldg(a.g_dn + R.act_e[s]);
+    const int ai = s / cpe;
+    const int q0 = (s % cpe) * srows;   // first row of the stage (from n0)
+    const int nq = min(srows, nr - q0);
+    const int slot0 = R.act_off[ai];
+    const int cnt = R.act_off[ai + 1] - slot0;   // > 1 only for a repeated expert id
+    const float g = __ldg(a.g_dn + R.act_e[ai]);
     const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
     const unsigned char *st = stage_base + (size_t)idx * stage_bytes;
-    const unsigned char *sbase = st + srows * rowb + (((int64_t)n0 * sclb) & 15);
+    const unsigned char *sbase = st + srows * rowb + (((int64_t)(n0 + q0) * sclb) & 15);
     for (int c = 0; c < cnt; ++c) {
       const int slot = slot0 + c;
       uint32_t xh[UPL][16];
@@ -1137,8 +1173,8 @@ __global__ void __launch_bounds__(32 * (CW + 1))
 #pragma unroll
         for (int i = 0; i < RPW; i += 2) {
           const int ra = cw + i * CW;
-          if (ra >= nr) break;   // warp-uniform
-          const int rb = ra + CW < nr ? ra + CW : ra;
+          if (ra >= nq) break;   // warp-uniform
+          const int rb = ra + CW < nq ? ra + CW : ra;
           float acc_a = 0.f, acc_b = 0.f;
 #pragma unroll
           for (int k = 0; k < UPL; ++k) {
@@ -1169,7 +1205,7 @@ __global__ void __launch_bounds__(32 * (CW + 1))
       const float tot = warp_reduce_many<RPW>(flat, lane);
       constexpr int SH = 5 - Log2<RPW>::value;
       const int r = cw + (lane >> SH) * CW;
-      if ((lane & ((1 << SH) - 1)) == 0 && r < nr) yk[(size_t)slot * nb + r] = tot * g * pss[slot];
+      if ((lane & ((1 << SH) - 1)) == 0 && r < nq) yk[(size_t)slot * nb + q0 + r] = tot * g * pss[slot];
     }
   }
   named_sync(2, nthreads_c);   // every y of this CTA is in yk
@@ -1274,13 +1310,14 @@ int launch_down_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
   const int64_t want = max64((int64_t)num_sms() * ctas_per_sm, ceil_div(a.H, kDownRows));
   const int nb = (int)ceil_div(a.H, want);
   const int64_t ctas = ceil_div(a.H, nb);
+  const int srows = (int)ceil_div(nb, kDownSplit);   // rows per stage
   const uint32_t stage_bytes =
-      align_up((uint32_t)(nb * (a.I / 2)) + span_bytes(nb * (a.I / 16)), 128);
+      align_up((uint32_t)(srows * (a.I / 2)) + span_bytes(srows * (a.I / 16)), 128);
   const Smem L = smem_layout(S, stage_bytes, CW, 0, n, (int)a.E, n * nb, (uint32_t)(n * a.I * 2));
   const int fit = resident_blocks(gemv_down_kernel<UPL, CW, S>, 32 * (CW + 1), L.total);
   if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
   return launch_pdl(gemv_down_kernel<UPL, CW, S>, dim3((unsigned)ctas), dim3(32 * (CW + 1)),
-                    L.total, s, a, stage_bytes, nb);
+                    L.total, s, a, stage_bytes, nb, srows);
 }
 
 }  // namespace
