@@ -26,6 +26,7 @@ __all__ = [
 ]
 
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
+WORKSPACE_ZERO_BYTES = 512   # head of a workspace that must be zero before first use
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libnvfp4moe.so")
 
@@ -169,8 +170,11 @@ def moe_nvfp4_workspace_size(T: int, H: int, I: int, E: int, K: int) -> int:
 
 
 def alloc_moe_workspace(T, H, I, E, K, device="cuda") -> torch.Tensor:
-    return torch.empty((moe_nvfp4_workspace_size(T, H, I, E, K),), dtype=torch.uint8,
-                       device=device)
+    """Workspace for moe_nvfp4_forward: its head (error flag and work counters) zeroed."""
+    ws = torch.empty((moe_nvfp4_workspace_size(T, H, I, E, K),), dtype=torch.uint8,
+                     device=device)
+    ws[:WORKSPACE_ZERO_BYTES].zero_()
+    return ws
 
 
 def moe_nvfp4_route(topk_ids: torch.Tensor, E: int):

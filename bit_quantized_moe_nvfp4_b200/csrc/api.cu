@@ -42,6 +42,7 @@ WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int
   };
   const size_t TK = (size_t)(T * K);
   L.flag = take(4);
+  L.work = take(8);   // zero before first use; every call leaves it zero
   L.n_active = take(4);
   L.counts = take(4 * (size_t)E);
   L.offsets = take(4 * (size_t)(E + 1));
@@ -139,6 +140,7 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   a.E = E;
   a.K = K;
   a.flag = reinterpret_cast<int32_t *>(ws + L.flag);
+  a.work = reinterpret_cast<int32_t *>(ws + L.work);
   a.n_active = reinterpret_cast<int32_t *>(ws + L.n_active);
   a.counts = reinterpret_cast<int32_t *>(ws + L.counts);
   a.offsets = reinterpret_cast<int32_t *>(ws + L.offsets);

@@ -422,26 +422,43 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
   pdl_launch_dependents();  // the down kernel may start routing and prefetching
 
   const int n_act = *R.n_act;
-  const int64_t units = (int64_t)n_act * I;
-  const int64_t U0 = units * blockIdx.x / gridDim.x, U1 = units * (blockIdx.x + 1) / gridDim.x;
+  // Work is handed out dynamically: chunk c is pair rows [j, j + P) of active expert c / cpe
+  // (j = (c % cpe) * P), claimed by the producers from the counter work[0], so CTAs that got
+  // their first stage late do less of it.  A producer holds at most one claimed chunk that
+  // it has not issued yet, and stops at its first claim past the end; the last producer to
+  // stop resets the counters.
+  const int cpe = (int)ceil_div(I, P);
+  const int total = n_act * cpe;
   const uint32_t rowb = (uint32_t)(H / 2), sclb = (uint32_t)(H / 16);
   const uint32_t span_stride = span_bytes(P * sclb);
+  __shared__ int s_unit[S], s_np[S];   // per stage: first unit (ai * I + j, -1 = no more), rows
 
   if (warp == 0) {
     // ------------------------------------------------ producer
     if (lane == 0) {
       int s = 0;
-      for (int64_t u = U0; u < U1; ++s) {
-        const int ai = (int)(u / I);
-        const int64_t j = u % I;
-        const int np = (int)min64(min64(P, I - j), U1 - u);
-        const int e = R.act_e[ai];
+      int next = atomicAdd(a.work, 1);   // claimed one chunk ahead: the atomic's round trip
+      for (;; ++s) {                     // overlaps the wait for a free stage
         const int idx = s % S;
         if (s >= S && (*(volatile int *)&s_abort || !mbar_wait(&empty[idx], ((s / S) - 1) & 1))) {
           if (!*(volatile int *)&s_abort) report_timeout(a.flag);
           *(volatile int *)&s_abort = 1;
           break;
         }
+        const int c = next;
+        if (c < total) next = atomicAdd(a.work, 1);
+        if (c >= total) {   // tell the consumers to stop (a plain arrive completes the phase)
+          s_unit[idx] = -1;
+          mbar_arrive(&full[idx]);
+          ++s;
+          break;
+        }
+        const int ai = c / cpe;
+        const int64_t j = (int64_t)(c % cpe) * P;
+        const int np = (int)min64(P, I - j);
+        const int e = R.act_e[ai];
+        s_unit[idx] = (int)(ai * I + j);
+        s_np[idx] = np;
         unsigned char *st = stage_base + (size_t)idx * stage_bytes;
         const int64_t rg = (int64_t)e * 2 * I + j;   // first gate row
         const int64_t ru = rg + I;                   // first up row
@@ -455,7 +472,12 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
         unsigned char *sc = st + 2 * P * rowb;
         bulk_g2s_span(sc, sblock, lg, np * sclb, &full[idx]);
         bulk_g2s_span(sc + span_stride, sblock, lu, np * sclb, &full[idx]);
-        u += np;
+      }
+      // this CTA claims nothing more: the last CTA to get here resets the counters
+      __threadfence();
+      if (atomicAdd(a.work + 1, 1) == (int)gridDim.x - 1) {
+        atomicExch(a.work, 0);
+        atomicExch(a.work + 1, 0);
       }
       // do not leave while copies into this CTA's shared memory may still be in flight
       const int issued = s;
@@ -467,40 +489,42 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
 
   if (warp == CW + 1) {
     // ------------------------------------------------ finalizer
-    int it = 0, cur_a = -1, slot0 = 0, cnt = 0;
+    // Each reduction slot carries its stage's first unit, rows and token group; a unit of -1
+    // marks the end.
+    int cur_a = -1, slot0 = 0, cnt = 0;
     float g = 0.f;
-    for (int64_t u = U0; u < U1;) {
-      const int ai = (int)(u / I);
-      const int64_t j = u % I;
-      const int np = (int)min64(min64(P, I - j), U1 - u);
+    for (int it = 0;; ++it) {
+      const int sl = it % kRedSlots;
+      if (!warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag)) break;
+      const float *rb = red + (size_t)sl * RS;
+      const int u = __float_as_int(rb[CW * RV + 4]);
+      if (u < 0) break;
+      const int np = __float_as_int(rb[CW * RV + 5]);
+      const int grp = __float_as_int(rb[CW * RV + 6]);
+      const int ai = u / (int)I;
+      const int64_t j = u % (int)I;
       if (ai != cur_a) {
         cur_a = ai;
         slot0 = R.act_off[ai];
         cnt = R.act_off[ai + 1] - slot0;
         g = __ldg(a.g_gu + R.act_e[ai]);
       }
-      for (int grp = 0; grp * NT < cnt; ++grp, ++it) {
-        const int nt = min(NT, cnt - grp * NT);
-        const int sl = it % kRedSlots;
-        const bool ok = warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag);
-        const float *rb = red + (size_t)sl * RS;
-        if (ok && lane < np * nt) {
-          const int pp = lane / nt, i = lane % nt;
-          float gs = 0.f, us = 0.f;
-          for (int w = 0; w < CW; ++w) {
-            gs += rb[w * RV + pp * NT + i];
-            us += rb[w * RV + (P + pp) * NT + i];
-          }
-          const float ps = rb[CW * RV + i];
-          const float gate = gs * g * ps;
-          const float up = us * g * ps;
-          const int slot = slot0 + grp * NT + i;
-          a.h[(int64_t)slot * I + j + pp] = __float2bfloat16_rn(silu_f32(gate) * up);
+      const int nt = min(NT, cnt - grp * NT);
+      if (lane < np * nt) {
+        const int pp = lane / nt, i = lane % nt;
+        float gs = 0.f, us = 0.f;
+        for (int w = 0; w < CW; ++w) {
+          gs += rb[w * RV + pp * NT + i];
+          us += rb[w * RV + (P + pp) * NT + i];
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&rfree[sl]);
+        const float ps = rb[CW * RV + i];
+        const float gate = gs * g * ps;
+        const float up = us * g * ps;
+        const int slot = slot0 + grp * NT + i;
+        a.h[(int64_t)slot * I + j + pp] = __float2bfloat16_rn(silu_f32(gate) * up);
       }
-      u += np;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfree[sl]);
     }
     return;
   }
@@ -515,7 +539,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
   for (int i = 0; i < NT; ++i) loaded_tok[i] = -1;
   int cur_a = -1, ngroups = 0, cnt = 0;
   int s = 0, it = 0;
-  if (NT == 1 && U0 < U1) {
+  if (NT == 1) {
     // One token: every pair is token 0, whose activations were loaded above; they are
     // scaled to f16 before the first stage arrives.
     float mx = 0.f;
@@ -539,18 +563,20 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
     loaded_tok[0] = 0;
     named_sync(1, nthreads_c);   // smax is rewritten by any later load
   }
-  for (int64_t u = U0; u < U1; ++s) {
-    const int ai = (int)(u / I);
-    const int64_t j = u % I;
-    const int np = (int)min64(min64(P, I - j), U1 - u);
+  for (;; ++s) {
     const int idx = s % S;
+    const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
+    const int u = have ? s_unit[idx] : -1;   // written before the producer's arrive
+    if (u < 0) break;                          // no more stages (or a wait gave up)
+    const int np = s_np[idx];
+    const int ai = u / (int)I;
+    const int64_t j = u % (int)I;
     const bool new_expert = ai != cur_a;
     if (new_expert) {
       cur_a = ai;
       cnt = R.act_off[ai + 1] - R.act_off[ai];
       ngroups = (cnt + NT - 1) / NT;
     }
-    const bool have = warp_wait(&full[idx], (s / S) & 1, &s_abort, a.flag);
     const unsigned char *st = stage_base + (size_t)idx * stage_bytes;
     const int64_t offg = j * sclb, offu = (I + j) * sclb;
     const unsigned char *spg = st + 2 * P * rowb + (offg & 15);
@@ -637,11 +663,21 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
       float *rb = red + (size_t)sl * RS;
       if ((lane & ((1 << SH) - 1)) == 0) rb[cw * RV + (lane >> SH)] = tot;
       if (cw == 0 && lane < NT) rb[CW * RV + lane] = pick<NT>(pscale, lane);
+      if (cw == 0 && lane == 0) {
+        rb[CW * RV + 4] = __int_as_float(u);
+        rb[CW * RV + 5] = __int_as_float(np);
+        rb[CW * RV + 6] = __int_as_float(grp);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rfull[sl]);
     }
-    u += np;
   }
+  // end marker for the finalizer
+  const int sl = it % kRedSlots;
+  if (it >= kRedSlots) warp_wait(&rfree[sl], ((it / kRedSlots) - 1) & 1, &s_abort, a.flag);
+  if (cw == 0 && lane == 0) red[(size_t)sl * RS + CW * RV + 4] = __int_as_float(-1);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&rfull[sl]);
 }
 
 // ================================================================== projections on mma.sync
@@ -1094,6 +1130,12 @@ __global__ void __launch_bounds__(32 * (CW + 1))
   const int nthreads_c = CW * 32;
   pdl_wait();   // h is written by the gate/up kernel
   pdl_launch_dependents();
+  // The gate/up grid is complete: its work counters are zero again (its last CTA reset
+  // them); rewriting them here keeps them zero even after a gate/up launch that failed.
+  if (blockIdx.x == 0 && cw == 0 && lane == 0) {
+    a.work[0] = 0;
+    a.work[1] = 0;
+  }
   const int n_valid = R.act_off[n_act];   // slots 0..n_valid-1 are the rows of h in use
   if (cw == 0 && lane == 0 && n_valid > 0) {
     const uint32_t bytes = (uint32_t)((int64_t)n_valid * I * 2);

@@ -21,6 +21,7 @@ struct MoeArgs {
   int64_t T, H, I, E, K;
   // workspace
   int32_t *flag;              // [1] error bits
+  int32_t *work;              // [2] work counters of the one-token gate/up kernel (zero)
   int32_t *n_active;          // [1]
   int32_t *counts;            // [E]
   int32_t *offsets;           // [E+1]
@@ -37,7 +38,7 @@ struct MoeArgs {
 
 // Workspace carve-up (byte offsets, each 256-aligned).
 struct WorkspaceLayout {
-  size_t flag, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, xscale, total;
+  size_t flag, work, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, xscale, total;
 };
 WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
 constexpr int kGatherPadRows = 256;

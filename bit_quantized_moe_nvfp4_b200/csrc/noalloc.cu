@@ -7,13 +7,15 @@
 // holds only the layer's own tensors, so it can neither allocate a workspace nor carve one
 // out of a buffer it owns.  The kernels are the ones moe_nvfp4_forward runs on its GEMV
 // path; only the scratch they write differs:
-//   h   [T*K, I] bf16   SwiGLU outputs, one row per routed pair    -> g_static_scratch
-//   y   [T*K, H] fp32   weighted expert outputs before the combine -> g_static_scratch
+//   work [2] int32      work counters of the one-token gate/up kernel -> g_static_scratch
+//   h   [T*K, I] bf16   SwiGLU outputs, one row per routed pair    -> g_static_scratch + 256
+//   y   [T*K, H] fp32   weighted expert outputs before the combine -> after h
 //   flag                error bits                                 -> the caller's pointer
-// Nothing in the scratch has to start at zero: the gate/up kernel writes every h row the
-// down kernel reads, the down kernel every y row the combine reads, and the flag is
-// overwritten by each call.  The array keeps the rows of
-// the last call after it ends.  There is ONE array per device, shared by every call on that
+// Of the scratch only the two work counters at its start (read by the one-token gate/up
+// kernel) have to be zero: they are zero when the library loads, and every call leaves them
+// zero.  Nothing else has to start at zero: the gate/up kernel writes every h row the down
+// kernel reads, the down kernel every y row the combine reads, and the flag is overwritten
+// by each call.  The array keeps the rows of the last call after it ends.  There is ONE array per device, shared by every call on that
 // device: calls on one stream are ordered and safe; calls that can overlap (different
 // streams or host threads on the same device) race on it.
 #include <mutex>
@@ -56,7 +58,8 @@ int static_scratch(unsigned char **base) {
   return NVFP4_OK;
 }
 
-// Bytes of h (rounded up to 256) and the offset of y inside the scratch.
+// Bytes of the counter block and of h (each rounded up to 256): h and y follow the counters.
+constexpr int64_t kStaticHead = 256;
 int64_t static_h_bytes(int64_t pairs, int64_t I) { return (pairs * I * 2 + 255) & ~int64_t(255); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -82,9 +85,9 @@ extern "C" int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *t
       !aligned16(s_gu) || !aligned16(s_dn) ||
       (reinterpret_cast<uintptr_t>(error_flag) & 3))
     return NVFP4_EINVAL;
-  // the fixed scratch bounds the batch: h (T*K*I bf16) and y (T*K*H fp32)
+  // the fixed scratch bounds the batch: counters, h (T*K*I bf16) and y (T*K*H fp32)
   if (!gemv_supported(T, H, I, K)) return NVFP4_ESHAPE;
-  if (static_h_bytes(T * K, I) + T * K * H * 4 > kStaticBytes) return NVFP4_ESHAPE;
+  if (kStaticHead + static_h_bytes(T * K, I) + T * K * H * 4 > kStaticBytes) return NVFP4_ESHAPE;
 
   unsigned char *base = nullptr;
   if (int s = static_scratch(&base)) return s;
@@ -106,8 +109,9 @@ extern "C" int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *t
   a.E = E;
   a.K = K;
   a.flag = error_flag;   // may be NULL: the kernels then skip the flag writes
-  a.h = reinterpret_cast<__nv_bfloat16 *>(base);
-  a.y = reinterpret_cast<float *>(base + static_h_bytes(T * K, I));
+  a.work = reinterpret_cast<int32_t *>(base);
+  a.h = reinterpret_cast<__nv_bfloat16 *>(base + kStaticHead);
+  a.y = reinterpret_cast<float *>(base + kStaticHead + static_h_bytes(T * K, I));
   if (int s = launch_gemv_gateup(a, stream)) return s;
   if (int s = launch_gemv_down(a, stream)) return s;
   return gemv_fused_combine(T) ? NVFP4_OK : launch_combine_pairs(a, stream);

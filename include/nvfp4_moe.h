@@ -121,10 +121,16 @@ NVFP4_API int nvfp4_cast_f32(const float *in, int64_t n, uint8_t *e4m3, uint8_t 
  * Limits: H % 64 == 0, I % 64 == 0, 1 <= K <= 16, E <= 1024, T*K < 2^31.
  * Alignment: x, w_gu, s_gu, w_dn, s_dn, out and workspace 16 bytes (EINVAL /
  * EWORKSPACE otherwise).
+ * Workspace: caller-owned device memory of moe_nvfp4_workspace_size bytes.  Its first
+ * NVFP4_WORKSPACE_ZERO_BYTES bytes hold the error flag and two work counters of the
+ * one-token kernels; they must be zero before the workspace's first call (cudaMemset), and
+ * every call leaves the counters zero again.  The rest needs no initialisation.  Calls that
+ * share a workspace must not overlap in time.
  * The call picks a memory-bound GEMV path for small T and a tensor-core grouped GEMM path
  * otherwise; both compute the same function.  It never synchronises with the host and
  * may be captured in a CUDA graph.
  * Errors: EINVAL, ESHAPE, EWORKSPACE (ws_bytes < moe_nvfp4_workspace_size), ECUDA. */
+#define NVFP4_WORKSPACE_ZERO_BYTES 512
 NVFP4_API size_t moe_nvfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
 
 NVFP4_API int moe_nvfp4_forward(const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w,
@@ -184,9 +190,10 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
 
 /* ---------------------------------------------------------------- fixed-scratch forward */
 
-/* Bytes of the fixed scratch of moe_nvfp4_forward_static: it holds T*K rows of I bf16 values
- * (rounded up to 256 bytes) and T*K rows of H fp32 values, so a call needs
- * roundup256(2*T*K*I) + 4*T*K*H <= 4 MiB (at H = 6144, I = 2048, K = 8: T <= 18). */
+/* Bytes of the fixed scratch of moe_nvfp4_forward_static: it holds 256 bytes of counters,
+ * T*K rows of I bf16 values (rounded up to 256 bytes) and T*K rows of H fp32 values, so a
+ * call needs 256 + roundup256(2*T*K*I) + 4*T*K*H <= 4 MiB (at H = 6144, I = 2048, K = 8:
+ * T <= 18). */
 #define NVFP4_STATIC_SCRATCH_BYTES 4194304
 
 /* The small-batch forward of moe_nvfp4_forward (its GEMV path: same kernels, same result)
@@ -199,8 +206,9 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
  *               moe_nvfp4_forward would (0, bit 0 = an id outside [0, E), bit 1 = a
  *               device-side wait gave up); overwritten by every call; 4-byte aligned.
  * Scratch: one array of NVFP4_STATIC_SCRATCH_BYTES per device, inside the library; no
- * call allocates or frees memory.  Nothing in it needs to start at zero.  It keeps the last
- * call's intermediate values after that call ends.  All calls on a device share it, so
+ * call allocates or frees memory.  Only its first 8 bytes (the work counters of the
+ * one-token kernels) must be zero at a call: they are zero when the library loads and every
+ * call leaves them zero.  It keeps the last call's intermediate values after that call ends.  All calls on a device share it, so
  * calls that can overlap in time (different streams, or different host threads, on the
  * same device) race; calls on one stream are ordered and safe.  The first call on each
  * device looks the array's address up (cudaGetSymbolAddress): make that first call before

@@ -167,6 +167,22 @@ def test_full_layer_decode(nv, full, path, T):
     _check_sampled(full, x, ids, w, out, tokens=[0, T - 1] if T > 1 else [0])
 
 
+def test_full_layer_single_token_calls_in_a_row(nv, full):
+    """Consecutive one-token calls on one workspace: the gate/up kernel hands out its
+    chunks from a counter in the workspace head, which every call must leave at zero for
+    the next one; each call is checked against the oracle."""
+    wl = synth.DECODE_T1
+    ws = nv.alloc_moe_workspace(1, wl.H, wl.I, wl.E, wl.K)
+    for n in range(3):
+        x = synth.activations_bf16(1, wl.H, 300 + n)
+        ids, w = synth.routing(1, wl.E, wl.K, seed=300 + n)
+        out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *full.dev, workspace=ws,
+                                   path=1)
+        torch.cuda.synchronize()
+        assert torch.all(ws[:nv.WORKSPACE_ZERO_BYTES].view(torch.int32)[1:] == 0)
+        _check_sampled(full, x, ids, w, out, tokens=[0])
+
+
 @pytest.mark.parametrize("path", [2, 0], ids=["gemm", "auto"])
 def test_full_layer_prefill(nv, full, path):
     wl = synth.PREFILL_T4096
