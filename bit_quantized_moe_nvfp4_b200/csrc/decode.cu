@@ -698,6 +698,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
 // activations are f16 with the per-token power-of-two scale, and the tensor core sums in
 // fp32.  This takes about a third of the instructions of a CUDA-core dot product per byte.
 constexpr int kGuWarps = 16;                  // compute warps
+constexpr int kGuFinal = 2;                   // finaliser warps (one per other reduction slot)
 constexpr int kGuMaxChunks = 3;               // 128-element chunks per warp: H <= 6144
 constexpr int kGuTok = 8;                     // token slots per group (MMA N)
 constexpr int kGuRedFloats = kGuWarps * 16 * kGuTok + 2 * kGuTok;   // per reduction slot
@@ -720,7 +721,7 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 }
 
 struct GuSmem {
-  uint32_t bars, stages, red, smax, ids, act_e, act_off, misc, hist, total;
+  uint32_t bars, stages, red, smax, ids, act_e, act_off, misc, hist, wts, total;
 };
 
 __host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, int n, int E) {
@@ -746,6 +747,8 @@ __host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, in
   o += 16;
   s.hist = o;
   o += 4 * E;
+  s.wts = o;   // [n] copy of topk_w (down: the finaliser weights each pair's y)
+  o += 4 * n;
   s.total = align_up(o, 128);
   return s;
 }
@@ -758,10 +761,13 @@ __host__ __device__ inline uint32_t gu_stage_bytes(int64_t Kd) {
   return 16 * gu_row_stride(Kd) + 2 * span_bytes(8 * (Kd / 16));
 }
 
-// blockDim = 32 * (kGuWarps + 2): warp 0 produces, warps 1..kGuWarps compute, the last warp
-// finalizes.
+// blockDim = 32 * (kGuWarps + 1 + kGuFinal): warp 0 produces, warps 1..kGuWarps compute,
+// the last kGuFinal warps finalize (finaliser f takes the reduction slots it with
+// it % kGuFinal == f, so each slot's barriers have one waiter, in order).  A warp's partial
+// sums sit token-major in its slot (token slot tk, tile row r at tk * 16 + r), so the
+// finalisers read them without bank conflicts.
 template <int MODE, int S>
-__global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
+__global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
     gemv_mma_kernel(MoeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ int s_abort;
@@ -801,6 +807,11 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
   // routing and the weight stream start before griddepcontrol.wait)
   const bool bad = cta_route(a.ids, n, E, R, hist);
   if (MODE == 0 && blockIdx.x == 0 && threadIdx.x == 0 && a.flag) *a.flag = bad ? kFlagBadId : 0;
+  float *wts = reinterpret_cast<float *>(smem + L.wts);
+  if (MODE == 1) {   // the pair weights, read once here instead of once per tile and output
+    for (int p = threadIdx.x; p < n; p += blockDim.x) wts[p] = __ldg(a.w + p);
+    __syncthreads();
+  }
   pdl_launch_dependents();  // the next kernel may start its prologue
 
   const int n_act = *R.n_act;
@@ -850,8 +861,9 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
     return;
   }
 
-  if (warp == CW + 1) {
-    // ------------------------------------------------ finalizer
+  if (warp > CW) {
+    // ------------------------------------------------ finalizers
+    const int fin = warp - CW - 1;
     int it = 0, cur_a = -1, slot0 = 0, cnt = 0;
     float gsc = 0.f;
     for (int64_t u = U0; u < U1; ++u) {
@@ -864,6 +876,7 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
         gsc = __ldg((MODE == 0 ? a.g_gu : a.g_dn) + R.act_e[ai]);
       }
       for (int grp = 0; grp * kGuTok < cnt; ++grp, ++it) {
+        if (it % kGuFinal != fin) continue;
         const int nt = min(kGuTok, cnt - grp * kGuTok);
         const int sl = it % kRedSlots;
         const bool ok = warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag);
@@ -871,12 +884,14 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
         if (MODE == 0) {
           for (int q = lane; ok && q < 8 * nt; q += 32) {
             const int tk = q >> 3, r = q & 7;   // token slot of the group, row pair
-            float gs = 0.f, us = 0.f;
-#pragma unroll 4
-            for (int w = 0; w < CW; ++w) {
-              gs += rb[w * 128 + r * 8 + tk];
-              us += rb[w * 128 + (8 + r) * 8 + tk];
+            float gp[4] = {0.f, 0.f, 0.f, 0.f}, up4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int w = 0; w < CW; ++w) {     // four chains, summed in a fixed order
+              gp[w & 3] += rb[w * 128 + tk * 16 + r];
+              up4[w & 3] += rb[w * 128 + tk * 16 + 8 + r];
             }
+            const float gs = (gp[0] + gp[1]) + (gp[2] + gp[3]);
+            const float us = (up4[0] + up4[1]) + (up4[2] + up4[3]);
             const float ps = rb[CW * 128 + tk];
             const float gate = gs * gsc * ps, up = us * gsc * ps;
             const int slot = slot0 + grp * kGuTok + tk;
@@ -885,12 +900,13 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
         } else {
           for (int q = lane; ok && q < 16 * nt; q += 32) {
             const int tk = q >> 4, r = q & 15;  // token slot of the group, output row
-            float ys = 0.f;
-#pragma unroll 4
-            for (int w = 0; w < CW; ++w) ys += rb[w * 128 + r * 8 + tk];
+            float yp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int w = 0; w < CW; ++w) yp[w & 3] += rb[w * 128 + tk * 16 + r];
+            const float ys = (yp[0] + yp[1]) + (yp[2] + yp[3]);
             const float ps = rb[CW * 128 + tk];
             const int pair = __float_as_int(rb[CW * 128 + kGuTok + tk]);
-            a.y[(int64_t)pair * H + j + r] = ys * gsc * ps * __ldg(a.w + pair);
+            a.y[(int64_t)pair * H + j + r] = ys * gsc * ps * wts[pair];
           }
         }
         __syncwarp();
@@ -1027,10 +1043,11 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 2), 1)
       }
       const int sl = it % kRedSlots;
       if (it >= kRedSlots) warp_wait(&rfree[sl], ((it / kRedSlots) - 1) & 1, &s_abort, a.flag);
-      float *rb = red + (size_t)sl * kGuRedFloats + cw * 128;
-      *reinterpret_cast<float2 *>(rb + g * 8 + 2 * t) = make_float2(d0[0] + d1[0], d0[1] + d1[1]);
-      *reinterpret_cast<float2 *>(rb + (8 + g) * 8 + 2 * t) =
-          make_float2(d0[2] + d1[2], d0[3] + d1[3]);
+      float *rb = red + (size_t)sl * kGuRedFloats + cw * 128;   // token-major: tk * 16 + row
+      rb[(2 * t) * 16 + g] = d0[0] + d1[0];
+      rb[(2 * t + 1) * 16 + g] = d0[1] + d1[1];
+      rb[(2 * t) * 16 + 8 + g] = d0[2] + d1[2];
+      rb[(2 * t + 1) * 16 + 8 + g] = d0[3] + d1[3];
       if (cw == 0 && t == 0) {
         red[(size_t)sl * kGuRedFloats + CW * 128 + g] = pscale;
         red[(size_t)sl * kGuRedFloats + CW * 128 + kGuTok + g] = __int_as_float(mypair);
@@ -1330,9 +1347,9 @@ template <int MODE, int S>
 int launch_mma_cfg(const MoeArgs &a, cudaStream_t s) {
   const int n = (int)(a.T * a.K);
   const GuSmem L = gu_smem_layout(S, gu_stage_bytes(MODE == 0 ? a.H : a.I), n, (int)a.E);
-  const int fit = resident_blocks(gemv_mma_kernel<MODE, S>, 32 * (kGuWarps + 2), L.total);
+  const int fit = resident_blocks(gemv_mma_kernel<MODE, S>, 32 * (kGuWarps + 1 + kGuFinal), L.total);
   if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
-  return launch_pdl(gemv_mma_kernel<MODE, S>, dim3(num_sms()), dim3(32 * (kGuWarps + 2)),
+  return launch_pdl(gemv_mma_kernel<MODE, S>, dim3(num_sms()), dim3(32 * (kGuWarps + 1 + kGuFinal)),
                     L.total, s, a);
 }
 
