@@ -753,10 +753,11 @@ __host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, in
   return s;
 }
 
-// Stage geometry for a reduction length Kd: 16 packed rows at a stride of Kd/2 + 16 bytes
-// (the pad spreads the rows over the shared-memory banks), then the block-scale runs of rows
+// Stage geometry for a reduction length Kd: 16 packed rows at a stride of Kd/2 bytes (rows
+// 0..7 and 8..15 each arrive with one bulk copy: per-row copies with a bank-spreading pad
+// were slower, the copy count per tile being the limit), then the block-scale runs of rows
 // 0..7 and 8..15.
-__host__ __device__ inline uint32_t gu_row_stride(int64_t Kd) { return (uint32_t)(Kd / 2 + 16); }
+__host__ __device__ inline uint32_t gu_row_stride(int64_t Kd) { return (uint32_t)(Kd / 2); }
 __host__ __device__ inline uint32_t gu_stage_bytes(int64_t Kd) {
   return 16 * gu_row_stride(Kd) + 2 * span_bytes(8 * (Kd / 16));
 }
@@ -846,11 +847,8 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
         const uint32_t span_g = (uint32_t)(((lg + 8 * sclb + 15) & ~15ll) - (lg & ~15ll));
         const uint32_t span_u = (uint32_t)(((lu + 8 * sclb + 15) & ~15ll) - (lu & ~15ll));
         mbar_arrive_expect_tx(&full[idx], 16u * rowb + span_g + span_u);
-#pragma unroll 1
-        for (int r = 0; r < 8; ++r) {
-          bulk_g2s(st + r * rstride, wblock + (lr0 + r) * rowb, rowb, &full[idx]);
-          bulk_g2s(st + (8 + r) * rstride, wblock + (lr1 + r) * rowb, rowb, &full[idx]);
-        }
+        bulk_g2s(st, wblock + lr0 * rowb, 8 * rowb, &full[idx]);            // rows 0..7
+        bulk_g2s(st + 8 * rstride, wblock + lr1 * rowb, 8 * rowb, &full[idx]);   // 8..15
         bulk_g2s_span(st + scl_off, sblock, lg, 8 * sclb, &full[idx]);
         bulk_g2s_span(st + scl_off + span_stride, sblock, lu, 8 * sclb, &full[idx]);
       }
