@@ -51,6 +51,21 @@ def test_small_layer_many_shapes(nv, path, T):
 
 
 @pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
+def test_batch_sizes_alternating(nv, path):
+    """Larger, smaller, then larger batches again on the same kernels: each launch needs
+    its own amount of shared memory, and a smaller call must not leave a kernel unable to
+    launch a larger one."""
+    E, H, I, K = 37, 192, 128, 4
+    layer = Layer(E, H, I, seed=21)
+    for n, T in enumerate([40, 3, 40, 9]):
+        x = synth.activations_bf16(T, H, 50 + n)
+        ids, w = synth.routing(T, E, K, seed=50 + n)
+        out = run(nv, layer, x, ids, w, path)
+        ref, ref64, _ = layer.oracle_forward(x, ids, w)
+        compare_moe(out, ref, ref64)
+
+
+@pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
 def test_edge_cases(nv, path):
     """One expert takes every token, most experts are empty, a zero token, a repeated id
     within a token, and an out-of-range id (contributes nothing, raises the flag)."""
