@@ -685,11 +685,11 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
 // (f16 x f16 -> fp32): M = 16 weight rows of one expert, N = 8 token slots, K = 16.
 //   MODE 0, gate/up: rows = gate rows j..j+7 and up rows j..j+7; the activations are x;
 //           result h[slot, j+r] = bf16( silu(g_gu * gate_r) * g_gu * up_r )  (SwiGLU)
-//   MODE 1, down:    rows = output rows r0..r0+15; the activations are the h rows of the
-//           expert's slots; result y[pair, r0+r] = w[pair] * g_dn * (W_dn h)_r, combined
-//           over k afterwards (combine.cu)
-// A unit is one such 16-row tile; each CTA takes a contiguous range of units in expert
-// order, so an expert's activations are loaded once per CTA.  Since a dot product may sum its terms in any order, the K index of the MMA is
+//   MODE 1, down:    rows = output rows r0..r0+31 (two M-tiles); the activations are the h
+//           rows of the expert's slots; result y[pair, r0+r] = w[pair] * g_dn * (W_dn h)_r,
+//           combined over k afterwards (combine.cu)
+// A unit is one such tile; each CTA takes a contiguous range of units in expert order, so an
+// expert's activations are loaded once per CTA.  Since a dot product may sum its terms in any order, the K index of the MMA is
 // mapped to memory so that each lane decodes only contiguous bytes: lane (g, t) (g = lane/4,
 // t = lane%4) owns elements 32t..32t+31 of every 128-element chunk, for weight rows g and
 // g+8 (A operand) and for token g (B operand); MMA i of a chunk takes elements
@@ -701,7 +701,15 @@ constexpr int kGuWarps = 16;                  // compute warps
 constexpr int kGuFinal = 2;                   // finaliser warps (one per other reduction slot)
 constexpr int kGuMaxChunks = 3;               // 128-element chunks per warp: H <= 6144
 constexpr int kGuTok = 8;                     // token slots per group (MMA N)
-constexpr int kGuRedFloats = kGuWarps * 16 * kGuTok + 2 * kGuTok;   // per reduction slot
+// Tile rows: 16 for gate/up (8 gate + 8 up rows, one MMA M-tile), 32 for down (two M-tiles:
+// the down tile is a third of a gate/up tile in bytes, and a tile's fixed cost -- the partial
+// sums, the finalisers, the barrier hand-offs -- is then paid once per 32 KB).
+__host__ __device__ constexpr int gu_mtiles(int mode) { return mode == 0 ? 1 : 2; }
+// Floats per reduction slot: each compute warp's partials (M-tiles x 16 rows x 8 tokens),
+// then the 8 tokens' 2^-p and pair indices.
+__host__ __device__ constexpr int gu_red_floats(int mode) {
+  return kGuWarps * 16 * gu_mtiles(mode) * kGuTok + 2 * kGuTok;
+}
 
 __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1,
                                               uint32_t a2, uint32_t a3, uint32_t b0,
@@ -724,7 +732,8 @@ struct GuSmem {
   uint32_t bars, stages, red, smax, ids, act_e, act_off, misc, hist, wts, total;
 };
 
-__host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, int n, int E) {
+__host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, int n, int E,
+                                                 int red_floats) {
   GuSmem s;
   uint32_t o = 0;
   s.bars = o;
@@ -733,7 +742,7 @@ __host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, in
   s.stages = o;
   o += stage_bytes * S;
   s.red = o;
-  o += 4 * kRedSlots * kGuRedFloats;
+  o += 4 * kRedSlots * red_floats;
   s.smax = o;
   o += 4 * kGuWarps * kGuTok;
   s.ids = o;
@@ -753,13 +762,13 @@ __host__ __device__ inline GuSmem gu_smem_layout(int S, uint32_t stage_bytes, in
   return s;
 }
 
-// Stage geometry for a reduction length Kd: 16 packed rows at a stride of Kd/2 bytes (rows
-// 0..7 and 8..15 each arrive with one bulk copy: per-row copies with a bank-spreading pad
-// were slower, the copy count per tile being the limit), then the block-scale runs of rows
-// 0..7 and 8..15.
+// Stage geometry for a reduction length Kd and rows = 16 x M-tiles: the packed rows at a
+// stride of Kd/2 bytes (each half of the tile arrives with one bulk copy: per-row copies with
+// a bank-spreading pad were slower, the copy count per tile being the limit), then the
+// block-scale runs of the two halves.
 __host__ __device__ inline uint32_t gu_row_stride(int64_t Kd) { return (uint32_t)(Kd / 2); }
-__host__ __device__ inline uint32_t gu_stage_bytes(int64_t Kd) {
-  return 16 * gu_row_stride(Kd) + 2 * span_bytes(8 * (Kd / 16));
+__host__ __device__ inline uint32_t gu_stage_bytes(int64_t Kd, int rows) {
+  return rows * gu_row_stride(Kd) + 2 * span_bytes((rows / 2) * (Kd / 16));
 }
 
 // blockDim = 32 * (kGuWarps + 1 + kGuFinal): warp 0 produces, warps 1..kGuWarps compute,
@@ -767,7 +776,8 @@ __host__ __device__ inline uint32_t gu_stage_bytes(int64_t Kd) {
 // it % kGuFinal == f, so each slot's barriers have one waiter, in order).  A warp's partial
 // sums sit token-major in its slot (token slot tk, tile row r at tk * 16 + r), so the
 // finalisers read them without bank conflicts.
-template <int MODE, int S>
+// MC: 128-element chunks per compute warp at most (reduction length <= 16 * 128 * MC).
+template <int MODE, int S, int MC>
 __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
     gemv_mma_kernel(MoeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -776,10 +786,13 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t H = a.H, I = a.I, K = a.K;
   const int64_t Kd = MODE == 0 ? H : I;          // reduction length
+  constexpr int MT = gu_mtiles(MODE);            // MMA M-tiles per tile
+  constexpr int RT = 16 * MT, HALF = RT / 2;     // rows per tile, rows per bulk copy
+  constexpr int RF = gu_red_floats(MODE);        // floats per reduction slot
   const int n = (int)(a.T * K);
   const int E = (int)a.E;
-  const uint32_t rstride = gu_row_stride(Kd), stage_bytes = gu_stage_bytes(Kd);
-  const GuSmem L = gu_smem_layout(S, stage_bytes, n, E);
+  const uint32_t rstride = gu_row_stride(Kd), stage_bytes = gu_stage_bytes(Kd, RT);
+  const GuSmem L = gu_smem_layout(S, stage_bytes, n, E, RF);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint64_t *empty = full + S;
   uint64_t *rfull = empty + S;
@@ -816,12 +829,12 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
   pdl_launch_dependents();  // the next kernel may start its prologue
 
   const int n_act = *R.n_act;
-  const int64_t upe = MODE == 0 ? I / 8 : H / 16;   // units per expert
+  const int64_t upe = MODE == 0 ? I / 8 : H / RT;   // units (tiles) per expert
   const int64_t units = (int64_t)n_act * upe;
   const int64_t U0 = units * blockIdx.x / gridDim.x, U1 = units * (blockIdx.x + 1) / gridDim.x;
   const uint32_t rowb = (uint32_t)(Kd / 2), sclb = (uint32_t)(Kd / 16);
-  const uint32_t scl_off = 16 * rstride;
-  const uint32_t span_stride = span_bytes(8 * sclb);
+  const uint32_t scl_off = RT * rstride;
+  const uint32_t span_stride = span_bytes(HALF * sclb);
 
   if (warp == 0) {
     // ------------------------------------------------ producer
@@ -837,20 +850,20 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
           break;
         }
         unsigned char *st = stage_base + (size_t)idx * stage_bytes;
-        // rows 0..7 and 8..15 of the tile, as row indices inside the expert's weight block
-        const int64_t lr0 = MODE == 0 ? (u % upe) * 8 : (u % upe) * 16;
-        const int64_t lr1 = MODE == 0 ? I + lr0 : lr0 + 8;
+        // the tile's two halves, as row indices inside the expert's weight block
+        const int64_t lr0 = MODE == 0 ? (u % upe) * 8 : (u % upe) * RT;
+        const int64_t lr1 = MODE == 0 ? I + lr0 : lr0 + HALF;
         const int64_t rows_pe = MODE == 0 ? 2 * I : H;
         const uint8_t *wblock = (MODE == 0 ? a.w_gu : a.w_dn) + (int64_t)e * rows_pe * rowb;
         const uint8_t *sblock = (MODE == 0 ? a.s_gu : a.s_dn) + (int64_t)e * rows_pe * sclb;
         const int64_t lg = lr0 * sclb, lu = lr1 * sclb;
-        const uint32_t span_g = (uint32_t)(((lg + 8 * sclb + 15) & ~15ll) - (lg & ~15ll));
-        const uint32_t span_u = (uint32_t)(((lu + 8 * sclb + 15) & ~15ll) - (lu & ~15ll));
-        mbar_arrive_expect_tx(&full[idx], 16u * rowb + span_g + span_u);
-        bulk_g2s(st, wblock + lr0 * rowb, 8 * rowb, &full[idx]);            // rows 0..7
-        bulk_g2s(st + 8 * rstride, wblock + lr1 * rowb, 8 * rowb, &full[idx]);   // 8..15
-        bulk_g2s_span(st + scl_off, sblock, lg, 8 * sclb, &full[idx]);
-        bulk_g2s_span(st + scl_off + span_stride, sblock, lu, 8 * sclb, &full[idx]);
+        const uint32_t span_g = (uint32_t)(((lg + HALF * sclb + 15) & ~15ll) - (lg & ~15ll));
+        const uint32_t span_u = (uint32_t)(((lu + HALF * sclb + 15) & ~15ll) - (lu & ~15ll));
+        mbar_arrive_expect_tx(&full[idx], (uint32_t)RT * rowb + span_g + span_u);
+        bulk_g2s(st, wblock + lr0 * rowb, HALF * rowb, &full[idx]);                 // first half
+        bulk_g2s(st + HALF * rstride, wblock + lr1 * rowb, HALF * rowb, &full[idx]);  // second
+        bulk_g2s_span(st + scl_off, sblock, lg, HALF * sclb, &full[idx]);
+        bulk_g2s_span(st + scl_off + span_stride, sblock, lu, HALF * sclb, &full[idx]);
       }
       const int issued = s;
       for (int t = max(0, issued - S); t < issued; ++t)
@@ -866,7 +879,7 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
     float gsc = 0.f;
     for (int64_t u = U0; u < U1; ++u) {
       const int ai = (int)(u / upe);
-      const int64_t j = MODE == 0 ? (u % upe) * 8 : (u % upe) * 16;   // first row / pair
+      const int64_t j = MODE == 0 ? (u % upe) * 8 : (u % upe) * RT;   // first row / pair
       if (ai != cur_a) {
         cur_a = ai;
         slot0 = R.act_off[ai];
@@ -878,32 +891,33 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
         const int nt = min(kGuTok, cnt - grp * kGuTok);
         const int sl = it % kRedSlots;
         const bool ok = warp_wait(&rfull[sl], (it / kRedSlots) & 1, &s_abort, a.flag);
-        const float *rb = red + (size_t)sl * kGuRedFloats;
+        const float *rb = red + (size_t)sl * RF;
         if (MODE == 0) {
           for (int q = lane; ok && q < 8 * nt; q += 32) {
             const int tk = q >> 3, r = q & 7;   // token slot of the group, row pair
             float gp[4] = {0.f, 0.f, 0.f, 0.f}, up4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
             for (int w = 0; w < CW; ++w) {     // four chains, summed in a fixed order
-              gp[w & 3] += rb[w * 128 + tk * 16 + r];
-              up4[w & 3] += rb[w * 128 + tk * 16 + 8 + r];
+              gp[w & 3] += rb[w * 128 * MT + tk * 16 + r];
+              up4[w & 3] += rb[w * 128 * MT + tk * 16 + 8 + r];
             }
             const float gs = (gp[0] + gp[1]) + (gp[2] + gp[3]);
             const float us = (up4[0] + up4[1]) + (up4[2] + up4[3]);
-            const float ps = rb[CW * 128 + tk];
+            const float ps = rb[CW * 128 * MT + tk];
             const float gate = gs * gsc * ps, up = us * gsc * ps;
             const int slot = slot0 + grp * kGuTok + tk;
             a.h[(int64_t)slot * I + j + r] = __float2bfloat16_rn(silu_f32(gate) * up);
           }
         } else {
-          for (int q = lane; ok && q < 16 * nt; q += 32) {
-            const int tk = q >> 4, r = q & 15;  // token slot of the group, output row
+          for (int q = lane; ok && q < RT * nt; q += 32) {
+            const int tk = q / RT, r = q % RT;  // token slot of the group, tile row
+            const int po = (r >> 4) * 128 + tk * 16 + (r & 15);   // M-tile, token, row
             float yp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-            for (int w = 0; w < CW; ++w) yp[w & 3] += rb[w * 128 + tk * 16 + r];
+            for (int w = 0; w < CW; ++w) yp[w & 3] += rb[w * 128 * MT + po];
             const float ys = (yp[0] + yp[1]) + (yp[2] + yp[3]);
-            const float ps = rb[CW * 128 + tk];
-            const int pair = __float_as_int(rb[CW * 128 + kGuTok + tk]);
+            const float ps = rb[CW * 128 * MT + tk];
+            const int pair = __float_as_int(rb[CW * 128 * MT + kGuTok + tk]);
             a.y[(int64_t)pair * H + j + r] = ys * gsc * ps * wts[pair];
           }
         }
@@ -920,21 +934,21 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
   const int g = lane >> 2, t = lane & 3;
   const int nchunk = (int)((Kd + 127) / 128);
   const int nthreads_c = CW * 32;
-  uint32_t xr[kGuMaxChunks][16];     // token g's activations (f16x2), chunk cw + CW*m
+  uint32_t xr[MC][16];     // token g's activations (f16x2), chunk cw + CW*m
   float pscale = 1.f;                // 2^-p of token g
   int loaded_tok = -2;               // activation row that lane group g holds
   int mypair = -1;                   // pair of slot g of the current group
   const __nv_bfloat16 *arow = MODE == 0 ? a.x : a.h;
 #pragma unroll
-  for (int m = 0; m < kGuMaxChunks; ++m)
+  for (int m = 0; m < MC; ++m)
 #pragma unroll
     for (int i = 0; i < 16; ++i) xr[m][i] = 0u;
   int cur_a = -1, ngroups = 0, cnt = 0;
   int s = 0, it = 0;
   for (int64_t u = U0; u < U1; ++u, ++s) {
     const int ai = (int)(u / upe);
-    const int64_t lr0 = MODE == 0 ? (u % upe) * 8 : (u % upe) * 16;
-    const int64_t lr1 = MODE == 0 ? I + lr0 : lr0 + 8;
+    const int64_t lr0 = MODE == 0 ? (u % upe) * 8 : (u % upe) * RT;
+    const int64_t lr1 = MODE == 0 ? I + lr0 : lr0 + HALF;
     const int idx = s % S;
     const bool new_expert = ai != cur_a;
     if (new_expert) {
@@ -964,7 +978,7 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
           float mx = 0.f;
           if (tok >= 0) {
 #pragma unroll
-            for (int m = 0; m < kGuMaxChunks; ++m) {
+            for (int m = 0; m < MC; ++m) {
               const int c = cw + CW * m;
               if (c < nchunk && c * 128 + 32 * t < Kd) {
                 uint4 v[4];
@@ -982,7 +996,7 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
           pscale = exp2i(-p);
           const float sp = exp2i(p);
 #pragma unroll
-          for (int m = 0; m < kGuMaxChunks; ++m) {
+          for (int m = 0; m < MC; ++m) {
             const int c = cw + CW * m;
             if (tok >= 0 && c < nchunk && c * 128 + 32 * t < Kd) {
               uint4 v[4];
@@ -996,42 +1010,57 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
           named_sync(1, nthreads_c);   // smax is rewritten by the next reload
         }
       }
-      // partial dot products over this warp's chunks: d[0..3] = rows (g, g+8) x tokens
-      // (2t, 2t+1) as the m16n8 accumulator layout has them; two chains for latency
-      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+      // partial dot products over this warp's chunks: per M-tile mt, d[0..3] = tile rows
+      // (16 mt + g, 16 mt + 8 + g) x tokens (2t, 2t+1) as the m16n8 accumulator layout has
+      // them; two chains per M-tile for latency
+      float d0[MT][4], d1[MT][4];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d0[mt][i] = d1[mt][i] = 0.f;
       if (have) {
 #pragma unroll
-        for (int m = 0; m < kGuMaxChunks; ++m) {
+        for (int m = 0; m < MC; ++m) {
           const int c = cw + CW * m;
           if (c >= nchunk) break;
           const bool lv = c * 128 + 32 * t < Kd;
-          uint4 wg = make_uint4(0u, 0u, 0u, 0u), wu = wg;
-          uint32_t sg = 0u, su = 0u;
-          if (lv) {
-            wg = *reinterpret_cast<const uint4 *>(st + g * rstride + c * 64 + 16 * t);
-            wu = *reinterpret_cast<const uint4 *>(st + (8 + g) * rstride + c * 64 + 16 * t);
-            sg = *reinterpret_cast<const unsigned short *>(sgb + g * sclb + c * 8 + 2 * t);
-            su = *reinterpret_cast<const unsigned short *>(sub + g * sclb + c * 8 + 2 * t);
-          }
-          // block scales as f16 pairs: blocks 2t (elements 0..15 of the lane) and 2t+1
-          const uint32_t sgh = e4m3x2_to_f16x2(sg), suh = e4m3x2_to_f16x2(su);
-          const uint32_t Sg[2] = {__byte_perm(sgh, 0, 0x1010), __byte_perm(sgh, 0, 0x3232)};
-          const uint32_t Su[2] = {__byte_perm(suh, 0, 0x1010), __byte_perm(suh, 0, 0x3232)};
-          const uint32_t wgw[4] = {wg.x, wg.y, wg.z, wg.w};
-          const uint32_t wuw[4] = {wu.x, wu.y, wu.z, wu.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {            // word q: elements 8q..8q+7, MMAs 2q, 2q+1
-            uint32_t hg[4], hu[4];
-            e2m1x8_to_f16x2x4(wgw[q], hg);
-            e2m1x8_to_f16x2x4(wuw[q], hu);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              hg[k] = hmul2_u32(hg[k], Sg[q >> 1]);
-              hu[k] = hmul2_u32(hu[k], Su[q >> 1]);
+          for (int mt = 0; mt < MT; ++mt) {
+            // tile rows R0 = 16 mt + g and R1 = R0 + 8; their scales sit in the run of the
+            // half (first HALF rows, or the rest) that holds them
+            const int R0 = 16 * mt + g, R1 = R0 + 8;
+            const unsigned char *s0 = 16 * mt >= HALF ? sub + (R0 - HALF) * sclb : sgb + R0 * sclb;
+            const unsigned char *s1 =
+                16 * mt + 8 >= HALF ? sub + (R1 - HALF) * sclb : sgb + R1 * sclb;
+            uint4 wg = make_uint4(0u, 0u, 0u, 0u), wu = wg;
+            uint32_t sg = 0u, su = 0u;
+            if (lv) {
+              wg = *reinterpret_cast<const uint4 *>(st + R0 * rstride + c * 64 + 16 * t);
+              wu = *reinterpret_cast<const uint4 *>(st + R1 * rstride + c * 64 + 16 * t);
+              sg = *reinterpret_cast<const unsigned short *>(s0 + c * 8 + 2 * t);
+              su = *reinterpret_cast<const unsigned short *>(s1 + c * 8 + 2 * t);
             }
-            // MMA 2q: elements 8q..8q+3; MMA 2q+1: elements 8q+4..8q+7
-            mma_16816_f16(d0, hg[0], hu[0], hg[1], hu[1], xr[m][4 * q], xr[m][4 * q + 1]);
-            mma_16816_f16(d1, hg[2], hu[2], hg[3], hu[3], xr[m][4 * q + 2], xr[m][4 * q + 3]);
+            // block scales as f16 pairs: blocks 2t (elements 0..15 of the lane) and 2t+1
+            const uint32_t sgh = e4m3x2_to_f16x2(sg), suh = e4m3x2_to_f16x2(su);
+            const uint32_t Sg[2] = {__byte_perm(sgh, 0, 0x1010), __byte_perm(sgh, 0, 0x3232)};
+            const uint32_t Su[2] = {__byte_perm(suh, 0, 0x1010), __byte_perm(suh, 0, 0x3232)};
+            const uint32_t wgw[4] = {wg.x, wg.y, wg.z, wg.w};
+            const uint32_t wuw[4] = {wu.x, wu.y, wu.z, wu.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {          // word q: elements 8q..8q+7, MMAs 2q, 2q+1
+              uint32_t hg[4], hu[4];
+              e2m1x8_to_f16x2x4(wgw[q], hg);
+              e2m1x8_to_f16x2x4(wuw[q], hu);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                hg[k] = hmul2_u32(hg[k], Sg[q >> 1]);
+                hu[k] = hmul2_u32(hu[k], Su[q >> 1]);
+              }
+              // MMA 2q: elements 8q..8q+3; MMA 2q+1: elements 8q+4..8q+7
+              mma_16816_f16(d0[mt], hg[0], hu[0], hg[1], hu[1], xr[m][4 * q], xr[m][4 * q + 1]);
+              mma_16816_f16(d1[mt], hg[2], hu[2], hg[3], hu[3], xr[m][4 * q + 2],
+                            xr[m][4 * q + 3]);
+            }
           }
         }
       }
@@ -1041,14 +1070,18 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
       }
       const int sl = it % kRedSlots;
       if (it >= kRedSlots) warp_wait(&rfree[sl], ((it / kRedSlots) - 1) & 1, &s_abort, a.flag);
-      float *rb = red + (size_t)sl * kGuRedFloats + cw * 128;   // token-major: tk * 16 + row
-      rb[(2 * t) * 16 + g] = d0[0] + d1[0];
-      rb[(2 * t + 1) * 16 + g] = d0[1] + d1[1];
-      rb[(2 * t) * 16 + 8 + g] = d0[2] + d1[2];
-      rb[(2 * t + 1) * 16 + 8 + g] = d0[3] + d1[3];
+      // this warp's partials: M-tile mt, token tk, row r at mt * 128 + tk * 16 + r
+      float *rb = red + (size_t)sl * RF + cw * 128 * MT;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        rb[mt * 128 + (2 * t) * 16 + g] = d0[mt][0] + d1[mt][0];
+        rb[mt * 128 + (2 * t + 1) * 16 + g] = d0[mt][1] + d1[mt][1];
+        rb[mt * 128 + (2 * t) * 16 + 8 + g] = d0[mt][2] + d1[mt][2];
+        rb[mt * 128 + (2 * t + 1) * 16 + 8 + g] = d0[mt][3] + d1[mt][3];
+      }
       if (cw == 0 && t == 0) {
-        red[(size_t)sl * kGuRedFloats + CW * 128 + g] = pscale;
-        red[(size_t)sl * kGuRedFloats + CW * 128 + kGuTok + g] = __int_as_float(mypair);
+        red[(size_t)sl * RF + CW * 128 * MT + g] = pscale;
+        red[(size_t)sl * RF + CW * 128 * MT + kGuTok + g] = __int_as_float(mypair);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rfull[sl]);
@@ -1355,13 +1388,14 @@ int launch_gateup_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
                     dim3(32 * (CW + 2)), L.total, s, a, stage_bytes);
 }
 
-template <int MODE, int S>
+template <int MODE, int S, int MC>
 int launch_mma_cfg(const MoeArgs &a, cudaStream_t s) {
   const int n = (int)(a.T * a.K);
-  const GuSmem L = gu_smem_layout(S, gu_stage_bytes(MODE == 0 ? a.H : a.I), n, (int)a.E);
-  const int fit = resident_blocks(gemv_mma_kernel<MODE, S>, 32 * (kGuWarps + 1 + kGuFinal), L.total);
+  const GuSmem L = gu_smem_layout(S, gu_stage_bytes(MODE == 0 ? a.H : a.I, 16 * gu_mtiles(MODE)),
+                                  n, (int)a.E, gu_red_floats(MODE));
+  const int fit = resident_blocks(gemv_mma_kernel<MODE, S, MC>, 32 * (kGuWarps + 1 + kGuFinal), L.total);
   if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
-  return launch_pdl(gemv_mma_kernel<MODE, S>, dim3(num_sms()), dim3(32 * (kGuWarps + 1 + kGuFinal)),
+  return launch_pdl(gemv_mma_kernel<MODE, S, MC>, dim3(num_sms()), dim3(32 * (kGuWarps + 1 + kGuFinal)),
                     L.total, s, a);
 }
 
@@ -1370,9 +1404,14 @@ int launch_mma_cfg(const MoeArgs &a, cudaStream_t s) {
 template <int MODE>
 int launch_mma(const MoeArgs &a, cudaStream_t s) {
   const int n = (int)(a.T * a.K);
-  const uint32_t sb = gu_stage_bytes(MODE == 0 ? a.H : a.I);
-  if (gu_smem_layout(3, sb, n, (int)a.E).total <= 227u * 1024u) return launch_mma_cfg<MODE, 3>(a, s);
-  return launch_mma_cfg<MODE, 2>(a, s);
+  const uint32_t sb = gu_stage_bytes(MODE == 0 ? a.H : a.I, 16 * gu_mtiles(MODE));
+  const bool three = gu_smem_layout(3, sb, n, (int)a.E, gu_red_floats(MODE)).total <= 227u * 1024u;
+  // one chunk per warp covers a reduction of 16 * 128 = 2048 (the down projection at
+  // I <= 2048): fewer registers held for the activations
+  if ((MODE == 0 ? a.H : a.I) <= 16 * 128)
+    return three ? launch_mma_cfg<MODE, 3, 1>(a, s) : launch_mma_cfg<MODE, 2, 1>(a, s);
+  return three ? launch_mma_cfg<MODE, 3, kGuMaxChunks>(a, s)
+               : launch_mma_cfg<MODE, 2, kGuMaxChunks>(a, s);
 }
 
 template <int UPL, int CW, int S>
