@@ -53,6 +53,20 @@ def test_workspace_queries(lib):
     assert lib.moe_nvfp4_workspace_size(0, 6144, 2048, 256, 8) == 0
 
 
+def test_workspace_zero_head(lib):
+    """The workspace head that must be zero before first use (error flag and the one-token
+    work counters) is the same size in the header and the Python binding, and every
+    workspace holds it."""
+    m = re.search(r"^#define NVFP4_WORKSPACE_ZERO_BYTES (\d+)", open(HEADER).read(), re.M)
+    assert m
+    import bit_quantized_moe_nvfp4_b200 as nv
+    assert nv.WORKSPACE_ZERO_BYTES == int(m.group(1))
+    lib.moe_nvfp4_workspace_size.restype = ctypes.c_size_t
+    lib.moe_nvfp4_workspace_size.argtypes = [ctypes.c_int64] * 5
+    for shape in ((1, 6144, 2048, 256, 8), (1, 64, 64, 1, 1), (37, 192, 128, 16, 4)):
+        assert lib.moe_nvfp4_workspace_size(*shape) >= nv.WORKSPACE_ZERO_BYTES
+
+
 def _fwd_argtypes(lib):
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f = lib.moe_nvfp4_forward_path
