@@ -11,14 +11,17 @@
 //                combine out[t] = bf16(sum_k w[t,k] y_k) in ascending k    (combine fused)
 //
 // Each CTA routes the tokens itself (histogram of the ids, exclusive scan, stable ranks) so
-// no separate routing launch is needed.  One producer warp streams the CTA's contiguous
-// share of expert rows into a shared-memory ring with 1-D bulk copies (cp.async.bulk,
-// completion counted on mbarriers); the consumer warps split the reduction dimension so
-// each lane owns a fixed slice of the activations, kept in registers as f16 with an exact
-// per-token power-of-two scale.  Lanes decode E2M1 pairs and E4M3 scales with the hardware
-// converts and accumulate with mixed-precision fma.rn.f32.f16 (f16 x f16 products are exact,
-// sums are fp32); partial sums are combined across lanes by recursive-halving shuffles and
-// across warps through shared memory.
+// no separate routing launch is needed.  One producer warp streams expert rows into a
+// shared-memory ring with 1-D bulk copies (cp.async.bulk, completion counted on mbarriers),
+// a few large copies per stage: the number of copies, more than their bytes, sets the pace.
+// With one token, the gate/up CTAs claim their row chunks from a counter in the workspace
+// (the last one resets it) and the down CTAs each own a slice of output rows for all
+// experts; with several tokens each CTA takes a contiguous range of tiles.  The compute
+// warps hold the activations as f16 with an exact per-token power-of-two scale; they decode
+// E2M1 pairs and E4M3 scales with the hardware converts and accumulate either with
+// mixed-precision fma.rn.f32.f16 (one token) or with mma.sync on f16 operands (several
+// tokens); f16 x f16 products are exact and sums fp32.  Partial sums are combined across
+// lanes by shuffles and across warps through shared memory.
 //
 // Activation scaling: x_t is multiplied by 2^p_t with p_t = 14 - floor(log2 max|x_t|) and
 // rounded to f16.  bf16 has 8 significant bits and f16 11, so this is exact for every
