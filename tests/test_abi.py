@@ -67,6 +67,15 @@ def test_workspace_zero_head(lib):
         assert lib.moe_nvfp4_workspace_size(*shape) >= nv.WORKSPACE_ZERO_BYTES
 
 
+def test_alloc_moe_workspace_zeroes_its_head(lib):
+    """The binding's allocator returns a workspace of the queried size whose head is zero
+    (host logic: checked with a CPU tensor)."""
+    import bit_quantized_moe_nvfp4_b200 as nv
+    ws = nv.alloc_moe_workspace(3, 192, 128, 16, 4, device="cpu")
+    assert ws.numel() == nv.moe_nvfp4_workspace_size(3, 192, 128, 16, 4)
+    assert int(ws[:nv.WORKSPACE_ZERO_BYTES].abs().sum()) == 0
+
+
 def _fwd_argtypes(lib):
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f = lib.moe_nvfp4_forward_path
