@@ -142,11 +142,13 @@ NVFP4_API int moe_nvfp4_forward(const __nv_bfloat16 *x, const int32_t *topk_ids,
 
 /* Paths of moe_nvfp4_forward_path. */
 #define NVFP4_PATH_AUTO 0     /* what moe_nvfp4_forward does */
-#define NVFP4_PATH_GEMV 1     /* dequant-fused grouped GEMV (CUDA cores), any T */
+#define NVFP4_PATH_GEMV 1     /* dequant-fused grouped GEMV (CUDA cores at T = 1, mma.sync for
+                                 T >= 2); T*K <= 1024, H <= 6144, I <= 6144 (3072 at T = 1) */
 #define NVFP4_PATH_GEMM 2     /* dequant-to-shared-memory grouped GEMM (tcgen05), any T */
 
 /* moe_nvfp4_forward with the path chosen by the caller (same arguments, same result up
- * to fp32 summation order).  Errors as moe_nvfp4_forward, plus EINVAL for a bad path. */
+ * to fp32 summation order).  Errors as moe_nvfp4_forward, plus EINVAL for a bad path and
+ * ESHAPE for a shape outside the GEMV limits when that path is asked for. */
 NVFP4_API int moe_nvfp4_forward_path(const __nv_bfloat16 *x, const int32_t *topk_ids,
                            const float *topk_w, int64_t T, int64_t H, int64_t I, int64_t E,
                            int64_t K, const uint8_t *w_gu, const uint8_t *s_gu,
@@ -215,7 +217,8 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
  * any stream capture begins on that device.
  * Errors: EINVAL (null or misaligned pointer, dimension <= 0), ESHAPE (the limits of
  * moe_nvfp4_forward, a batch whose h and y do not fit NVFP4_STATIC_SCRATCH_BYTES, or a
- * shape the GEMV path does not take: T*K > 1024, H > 6144 or I > 6144), ECUDA. */
+ * shape the GEMV path does not take: T*K > 1024, H > 6144, I > 6144, or I > 3072 with
+ * T = 1), ECUDA. */
 NVFP4_API int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *topk_ids,
                                        const float *topk_w, int64_t T, int64_t H, int64_t I,
                                        int64_t E, int64_t K, const uint8_t *w_gu,
