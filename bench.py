@@ -2,16 +2,21 @@
 """Benchmark of the NVFP4 routed-expert MoE layer on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode1|decode8|decode32|decode64|prefill|codec]
+                    [--workload all|prefill|decode1|decode8|decode32|decode64|codec]
 
 A step is one pass of the whole layer (route -> gate/up + SwiGLU -> down -> combine) over
-one batch.  The default workload is the single-token decode of the H=6144, I=2048, E=256,
-top-8 layer: every step routes a NEW token (synthetic x ~ N(0,1), router logits N(0,1),
-softmax top-8) to 8 of 256 experts whose NVFP4 weights (5.4 GB, N(0,0.02) bf16 quantized by
-the library) stay resident in HBM, so each step reads ~170 MB of expert bytes that are
-not in the 126 MB L2.  Steps are captured in a CUDA graph and timed with CUDA events.
+one batch of the H=6144, I=2048, E=256, top-8 layer whose NVFP4 weights (5.4 GB, N(0,0.02)
+bf16 quantized by the library) stay resident in HBM.  The headline line is the largest
+single-GPU configuration, prefill of T=4096 tokens with Zipf-like routing (x ~ N(0,1); expert
+e gets router-logit bias 1.5 ln(1/(e+1)) plus N(0,1) noise; top-8).  Every timed step routes
+a NEW batch, so the expert bytes it reads are not left in the 126 MB L2 by the step before.
+Steps are replayed from a CUDA graph and timed with CUDA events on the launching stream.
 
-Keys beyond the base contract: `roofline` (dominant kernel, live CUDA-event durations of
+With --workload all (the default, one GPU) the line also carries `sub_records`: decode of
+T = 1, 8, 32 and 64 tokens (HBM-bound GEMV path) and the whole-layer quantize / dequantize
+sweep, each timed the same way with its own step count, clock samples and roofline.
+
+Keys beyond the base contract: `roofline` (dominant kernel; live CUDA-event durations of
 each stage from a second, marked pass), `cpu_baseline` (the CPU oracle on a bounded
 sample, rank 0 at N=1), `e2e` (the same metric through the C ABI with pinned host
 buffers, copies inside the timed region), `clocks`, `gpu_launches`.
@@ -70,13 +75,18 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling in the background during the timed region."""
+    """nvidia-smi clock / throttle sampling in the background during the timed region.
+
+    Sampling starts `pre_s` seconds before the region; meanwhile `busy` (untimed replays of
+    the same work on `stream`) keeps the GPU under the region's load, so the samples taken
+    just before a short region describe the clocks it runs at."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_index: int, stream=None, busy=None, pre_s: float = 0.3):
+        self.gpu = physical_gpu(gpu_index)
+        self.stream, self.busy, self.pre_s = stream, busy, pre_s
         self.proc = None
 
     def __enter__(self):
@@ -87,7 +97,14 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.25)
+        t_end = time.perf_counter() + self.pre_s
+        if self.busy is not None:
+            with torch.cuda.stream(self.stream):
+                while time.perf_counter() < t_end:
+                    self.busy()
+                    self.stream.synchronize()
+        else:
+            time.sleep(self.pre_s)
         return self
 
     def __exit__(self, *exc):
@@ -117,6 +134,16 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_gpu(local_index: int) -> str:
+    """nvidia-smi's name for torch device `local_index` (CUDA_VISIBLE_DEVICES may remap)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        parts = [p.strip() for p in vis.split(",") if p.strip()]
+        if local_index < len(parts):
+            return parts[local_index]
+    return str(local_index)
 
 
 # ----------------------------------------------------------------------------- setup
@@ -166,164 +193,266 @@ def random_nvfp4_pool(pool, seed=11, i_rows=I):
     return pg, sg, g, pd, sd, g.copy()
 
 
-def cpu_baseline_decode(n_tokens=32, seed=7):
-    """The CPU oracle on a bounded sample: n_tokens single-token decode steps, each routed
-    to 8 of a pool of 16 experts."""
+def cpu_baseline(wl, n_tokens=24, seed=7):
+    """The CPU oracle on a bounded sample of the workload: n_tokens tokens of a batch routed
+    like `wl` (Zipf bias for prefill) to 8 of a pool of 16 experts, as one oracle call."""
     import oracle
     pool = 16
     weights = random_nvfp4_pool(pool)
-    ids, w = synth.routing(n_tokens, pool, K, seed=seed)
+    ids, w = synth.routing(n_tokens, pool, K, seed=seed, zipf_bias=wl.zipf_bias)
     x = synth.activations_bf16(n_tokens, H, seed)
     t0 = time.perf_counter()
-    for t in range(n_tokens):
-        oracle.moe_forward(x[t:t + 1], ids[t:t + 1], w[t:t + 1], *weights)
+    oracle.moe_forward(x, ids, w, *weights)
     total = time.perf_counter() - t0
     return {"value": n_tokens / total, "unit": "tokens/s", "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": f"{n_tokens} single-token decode steps of the H=6144 I=2048 top-8 layer "
-                      f"(fp64, {oracle.threads()} OpenMP threads)"}
+            "sample": f"{n_tokens} tokens of the {wl.name} workload (routing over a pool of "
+                      f"{pool} experts; fp64, {oracle.threads()} OpenMP threads)"}
 
 
 # ----------------------------------------------------------------------------- ours
+class Bench:
+    """One device, one resident layer: times workloads of the layer and the codec."""
+
+    def __init__(self, nv, args, rank, world, device):
+        self.nv, self.args, self.rank, self.world, self.device = nv, args, rank, world, device
+        self.peaks = load_peaks()
+        self.layer = None
+
+    def ensure_layer(self):
+        if self.layer is None:
+            self.layer = build_layer(self.nv, self.device)
+        return self.layer
+
+    def drop_layer(self):
+        self.layer = None
+        torch.cuda.empty_cache()
+
+    def layer_record(self, name, steps, warmup, main):
+        """Time `steps` steps of workload `name` (after `warmup` untimed steps)."""
+        nv, args, world, device = self.nv, self.args, self.world, self.device
+        peaks = self.peaks
+        wl = workload_of(name)
+        T = wl.T
+        layer = self.ensure_layer()
+        G = min(steps, args.graph_steps if T <= 64 else 2)   # steps per graph replay
+        n_b = max(G, warmup)
+        xs, ids, ws_ = make_batches(wl, n_b, seed=1000 + self.rank, device=device)
+        ws = nv.alloc_moe_workspace(T, H, I, E, K, device)
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        path = args.path
+
+        def step(i):
+            nv.moe_nvfp4_forward(xs[i], ids[i], ws_[i], *layer, out=out, workspace=ws,
+                                 path=path)
+
+        for i in range(warmup):
+            step(i % n_b)
+        torch.cuda.synchronize()
+
+        stream = torch.cuda.Stream(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            step(0)
+            stream.synchronize()
+            with torch.cuda.graph(graph, stream=stream):
+                for i in range(G):
+                    step(i)
+        reps, rem = divmod(steps, G)
+        tail_graph = None
+        if rem:
+            tail_graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(tail_graph, stream=stream):
+                for i in range(rem):
+                    step(i)
+        graph.replay()
+        torch.cuda.synchronize()
+
+        barrier(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device(), stream, graph.replay) as clk:
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(reps):
+                    graph.replay()
+                if tail_graph is not None:
+                    tail_graph.replay()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+        ms_step = ms_total / steps
+
+        # marked pass: per-stage durations from events between the kernels
+        n_mark = min(G, 64)
+        marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_mark)]
+        for m in marks:          # torch creates the CUDA event on its first record
+            for e in m:
+                e.record()
+        torch.cuda.synchronize()
+        mgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(mgraph, stream=stream):
+                for i in range(n_mark):
+                    nv.moe_nvfp4_forward_profiled(xs[i], ids[i], ws_[i], *layer, out, ws,
+                                                  marks[i], path=path)
+            mgraph.replay()
+        torch.cuda.synchronize()
+        stages = {n: statistics.mean(m[j].elapsed_time(m[j + 1]) for m in marks)
+                  for j, n in enumerate(["route", "gate_up", "down", "combine"])}
+        marked_step = statistics.mean(m[0].elapsed_time(m[4]) for m in marks)
+
+        uniq = statistics.mean(len(set(ids[i].flatten().tolist())) for i in range(G))
+        bytes_step = uniq * EXPERT_BYTES
+        flops_step = 2 * T * K * (3 * H * I)
+        value = T * steps * world / (ms_total / 1e3)
+
+        gemv = path == 1 or (path == 0 and T <= 64)
+        if gemv:   # HBM-bound: the gate/up GEMV streams 2/3 of the expert bytes
+            gu_ms = stages["gate_up"]
+            achieved = uniq * GATEUP_BYTES_PER_EXPERT / (gu_ms / 1e3) / 1e9
+            kname = "gemv_gateup_kernel" if T == 1 else "gemv_mma_kernel<0>"
+            roof = {"kernel": kname + " (gate/up + SwiGLU)", "bound": "hbm",
+                    "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(kname),
+                    "algorithmic_bytes": uniq * GATEUP_BYTES_PER_EXPERT,
+                    "peak_source": peaks["source"] + " (burst copy)"}
+            launches = 2 if T == 1 else 3
+        else:
+            gu_ms = stages["gate_up"]
+            fl = 2 * T * K * (2 * I * H)
+            achieved = fl / (gu_ms / 1e3) / 1e12
+            pk = peaks["bf16_tflops"]
+            roof = {"kernel": "gemm_kernel mode 0 (tcgen05 grouped GEMM + SwiGLU)",
+                    "bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                    "frac": achieved / pk, "traffic": measured_traffic("gemm_kernel_gateup"),
+                    "algorithmic_flops": fl,
+                    "peak_source": peaks["source"] + " (cuBLAS bf16 burst; the f16 MMA has the "
+                                                     "same dense rate)"}
+            launches = 5    # route, gather, gate/up GEMM, down GEMM, combine
+
+        e2e = run_e2e(nv, layer, wl, args, device, ws, path)
+        rec = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16/bf16 products of NVFP4 weights, f32 accumulation",
+            "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) bf16 weights quantized to NVFP4)",
+            "config": {"workload": wl.name if E == 256 else wl.name.replace("E=256", f"E={E}"),
+                       "T": T, "H": H, "I": I, "E": E, "K": K,
+                       "weights": "NVFP4 (E2M1 + E4M3 per 16 + fp32 per tensor), "
+                                  f"{E * EXPERT_BYTES / 1e9:.2f} GB resident",
+                       "l2": "inputs larger than L2: every step routes new tokens over 5.4 GB "
+                             "of expert weights (>126 MB L2)",
+                       "timing": f"CUDA graph of {G} steps replayed, CUDA events",
+                       "path": {0: "auto", 1: "gemv", 2: "gemm"}[path],
+                       "parallelism": f"{world} independent replica(s), no data-path "
+                                      "collective"},
+            "hbm_gbs_step": bytes_step / (ms_step / 1e3) / 1e9,
+            "tflops_step": flops_step / (ms_step / 1e3) / 1e12,
+            "unique_experts_per_step": uniq,
+            "stages_ms": stages, "marked_step_ms": marked_step,
+            "roofline": roof,
+            "e2e": e2e,
+            "gpu_launches": launches * steps,
+            "clocks": clk.summary(),
+        }
+        if main and self.rank == 0 and world == 1 and not args.no_cpu_baseline:
+            rec["cpu_baseline"] = cpu_baseline(wl, args.cpu_tokens)
+        del graph, tail_graph, mgraph, xs, ids, ws_, ws
+        torch.cuda.empty_cache()
+        return rec
+
+    def codec_record(self, steps, warmup):
+        """Whole-layer quantize + dequantize of all 256 experts (gate/up and down)."""
+        nv, world, device, peaks = self.nv, self.world, self.device, self.peaks
+        wl = synth.CODEC_LAYER
+        xs = {}
+        for proj, shape in (("w_gu", (2 * I, H)), ("w_dn", (H, I))):
+            x = torch.empty((E,) + shape, dtype=torch.bfloat16, device=device)
+            for e in range(E):
+                x[e] = synth.normal_bf16(shape, wl.seed, proj, e, std=0.02, device=device,
+                                         outlier_p=wl.outlier_p)
+            xs[proj] = x
+        outs = {p: nv.nvfp4_quantize(x) for p, x in xs.items()}
+        qws = {p: torch.zeros((nv.nvfp4_quantize_workspace_size(*x.shape),), dtype=torch.uint8,
+                              device=device) for p, x in xs.items()}
+        deq = {p: torch.empty_like(x) for p, x in xs.items()}
+        elts = sum(x.numel() for x in xs.values())
+        stream = torch.cuda.current_stream(device)
+
+        def q():
+            for p, x in xs.items():
+                nv.nvfp4_quantize(x, *outs[p], workspace=qws[p])
+
+        def d():
+            for p in xs:
+                nv.nvfp4_dequantize(*outs[p], out=deq[p])
+
+        res = {}
+        for name, fn in (("quantize", q), ("dequantize", d)):
+            for _ in range(warmup):
+                fn()
+            torch.cuda.synchronize()
+            barrier(world)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(torch.cuda.current_device(), stream, fn) as clk:
+                torch.cuda.synchronize()
+                e0.record(stream)
+                for _ in range(steps):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+            barrier(world)
+            ms = max_over_ranks(e0.elapsed_time(e1), world, device) / steps
+            gbs = elts * 2.5625 / (ms / 1e3) / 1e9
+            kern = name + "_kernel"
+            res[name] = {
+                "ms_per_layer": ms, "GB/s": gbs,
+                "roofline": {"kernel": kern, "bound": "hbm", "achieved": gbs,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"],
+                             "traffic": measured_traffic(kern),
+                             "algorithmic_bytes": elts * 2.5625,
+                             "peak_source": peaks["source"] + " (burst copy)"},
+                "clocks": clk.summary(),
+                # one launch per projection per layer
+                "gpu_launches": 2 * steps}
+        del xs, outs, deq, qws
+        torch.cuda.empty_cache()
+        return {"metric": "NVFP4 codec GB/s (whole layer)", "unit": "GB/s",
+                "value": res["quantize"]["GB/s"], "steps": steps, "warmup": warmup,
+                "higher_is_better": True, "dtype": "f32 (codec arithmetic), u8 codes",
+                "config": {"workload": wl.name, "elements": elts,
+                           "bytes_per_element": "2 (bf16) + 0.5625 (codes + scales)",
+                           "l2": "inputs (19.3 GB bf16) larger than L2"},
+                "roofline": res["quantize"]["roofline"],
+                "quantize": res["quantize"], "dequantize": res["dequantize"]}
+
+
+SUB_DECODE_STEPS = {"decode1": 4096, "decode8": 1024, "decode32": 512, "decode64": 256}
+
+
 def run_ours(args, rank, world, device):
     import bit_quantized_moe_nvfp4_b200 as nv
-    peaks = load_peaks()
-    wl = workload_of(args.workload)
+    b = Bench(nv, args, rank, world, device)
     if args.workload == "codec":
-        return run_codec(args, nv, rank, world, device, peaks)
-    T = wl.T
-    layer = build_layer(nv, device)
-    # distinct token batches; a graph of G steps is replayed to cover K steps exactly
-    K_steps, W = args.steps, args.warmup
-    G = min(K_steps, args.graph_steps if T <= 64 else 2)
-    n_b = max(G, W)
-    xs, ids, ws_ = make_batches(wl, n_b, seed=1000 + rank, device=device)
-    ws = nv.alloc_moe_workspace(T, H, I, E, K, device)
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-    path = args.path
-
-    def step(i):
-        nv.moe_nvfp4_forward(xs[i], ids[i], ws_[i], *layer, out=out, workspace=ws, path=path)
-
-    for i in range(W):
-        step(i % n_b)
-    torch.cuda.synchronize()
-
-    # graph of G steps (same kernels, same order as eager calls)
-    stream = torch.cuda.Stream(device)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        step(0)
-        stream.synchronize()
-        with torch.cuda.graph(graph, stream=stream):
-            for i in range(G):
-                step(i)
-    reps, rem = divmod(K_steps, G)
-    tail_graph = None
-    if rem:
-        tail_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(tail_graph, stream=stream):
-            for i in range(rem):
-                step(i)
-    graph.replay()
-    torch.cuda.synchronize()
-
-    barrier(world)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda.synchronize()
-        ev0.record(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(reps):
-                graph.replay()
-            if tail_graph is not None:
-                tail_graph.replay()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms_total = ev0.elapsed_time(ev1)
-    ms_total = max_over_ranks(ms_total, world, device)
-    ms_step = ms_total / K_steps
-
-    # marked pass: per-stage durations from events between the kernels
-    n_mark = min(G, 64)
-    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_mark)]
-    for m in marks:          # torch creates the CUDA event on its first record
-        for e in m:
-            e.record()
-    torch.cuda.synchronize()
-    mgraph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(mgraph, stream=stream):
-            for i in range(n_mark):
-                nv.moe_nvfp4_forward_profiled(xs[i], ids[i], ws_[i], *layer, out, ws, marks[i],
-                                              path=path)
-        mgraph.replay()
-    torch.cuda.synchronize()
-    stages = {n: statistics.mean(m[j].elapsed_time(m[j + 1]) for m in marks)
-              for j, n in enumerate(["route", "gate_up", "down", "combine"])}
-    marked_step = statistics.mean(m[0].elapsed_time(m[4]) for m in marks)
-
-    # algorithmic work of the timed steps
-    counts = []
-    for i in range(G):
-        counts.append(len(set(ids[i].flatten().tolist())))
-    uniq = statistics.mean(counts)
-    bytes_step = uniq * EXPERT_BYTES
-    flops_step = 2 * T * K * (3 * H * I)
-    tokens_total = T * K_steps * world
-    value = tokens_total / (ms_total / 1e3)
-
-    gemv = path == 1 or (path == 0 and T <= 64)
-    if gemv:   # HBM-bound: the gate/up GEMV streams 2/3 of the expert bytes
-        gu_ms = stages["gate_up"]
-        achieved = uniq * GATEUP_BYTES_PER_EXPERT / (gu_ms / 1e3) / 1e9
-        kname = "gemv_gateup_kernel" if T == 1 else "gemv_mma_kernel<0>"
-        roof = {"kernel": kname + " (gate/up + SwiGLU)", "bound": "hbm",
-                "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(kname),
-                "algorithmic_bytes": uniq * GATEUP_BYTES_PER_EXPERT,
-                "peak_source": peaks["source"] + " (burst copy)"}
-    else:
-        gu_ms = stages["gate_up"]
-        fl = 2 * T * K * (2 * I * H)
-        achieved = fl / (gu_ms / 1e3) / 1e12
-        pk = peaks["bf16_tflops"]
-        roof = {"kernel": "gemm_gateup (tcgen05 grouped GEMM + SwiGLU)", "bound": "tensor",
-                "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
-                "traffic": None, "algorithmic_flops": fl,
-                "peak_source": peaks["source"] + " (cuBLAS bf16 burst)"}
-
-    # end to end through the C ABI with pinned host buffers
-    e2e = run_e2e(nv, layer, wl, args, device, ws, path)
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": K_steps, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4 weights; f16/bf16 products, f32 accumulation",
-        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) bf16 weights quantized to NVFP4)",
-        "config": {"workload": wl.name if E == 256 else wl.name.replace("E=256", f"E={E}"),
-                   "T": T, "H": H, "I": I, "E": E, "K": K,
-                   "weights": "NVFP4 (E2M1 + E4M3 per 16 + fp32 per tensor), "
-                              f"{E * EXPERT_BYTES / 1e9:.2f} GB resident",
-                   "l2": "inputs larger than L2: every step routes new tokens over 5.4 GB of "
-                         "expert weights (>126 MB L2)",
-                   "timing": f"CUDA graph of {G} steps replayed, CUDA events",
-                   "path": {0: "auto", 1: "gemv", 2: "gemm"}[path],
-                   "parallelism": f"{world} independent replica(s), no data-path collective"},
-        "hbm_gbs_step": bytes_step / (ms_step / 1e3) / 1e9,
-        "tflops_step": flops_step / (ms_step / 1e3) / 1e12,
-        "unique_experts_per_step": uniq,
-        "stages_ms": stages, "marked_step_ms": marked_step,
-        "roofline": roof,
-        "e2e": e2e,
-        # GEMV: gate/up + down (+ combine for T > 1); GEMM: route, gather, 2 GEMMs, combine
-        "gpu_launches": ((2 if T == 1 else 3) if gemv else 5) * K_steps,
-        "clocks": clk.summary(),
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_decode(args.cpu_tokens)
+        rec = b.codec_record(args.steps, args.warmup)
+        rec.update({"n_gpus": world, "scaling": "weak", "vs_baseline": None,
+                    "data": "synthetic", "ms_per_step": rec["quantize"]["ms_per_layer"],
+                    "clocks": rec["quantize"]["clocks"],
+                    "gpu_launches": rec["quantize"]["gpu_launches"]})
+        return rec
+    main = "prefill" if args.workload == "all" else args.workload
+    line = b.layer_record(main, args.steps, args.warmup, main=True)
+    if args.workload == "all" and world == 1 and not args.no_sub_records:
+        subs = []
+        for name, n in SUB_DECODE_STEPS.items():
+            subs.append(b.layer_record(name, max(n, args.steps), args.warmup, main=False))
+        b.drop_layer()
+        subs.append(b.codec_record(max(3, min(args.steps, 8)), args.warmup))
+        line["sub_records"] = subs
     return line
 
 
@@ -331,7 +460,7 @@ def run_e2e(nv, layer, wl, args, device, ws, path):
     """Same metric through the public API with host buffers: per step, copy the step's
     x / ids / weights from pinned host memory, run the layer, copy the output back."""
     T = wl.T
-    n = max(1, min(args.e2e_steps, 256 if T <= 64 else 4))
+    n = max(1, min(args.e2e_steps, 256 if T <= 64 else 8))
     xs = synth.activations_bf16(n * T, H, 77).view(n, T, H).pin_memory()
     ids, w = synth.routing(n * T, E, K, seed=77, zipf_bias=wl.zipf_bias)
     ids = ids.view(n, T, K).pin_memory()
@@ -363,74 +492,25 @@ def run_e2e(nv, layer, wl, args, device, ws, path):
             "h2d_bytes_per_step": T * H * 2 + T * K * 4 * 2, "d2h_bytes_per_step": T * H * 2}
 
 
-def run_codec(args, nv, rank, world, device, peaks):
-    """Whole-layer quantize + dequantize of all 256 experts (gate/up and down)."""
-    wl = synth.CODEC_LAYER
-    xs = {}
-    for proj, shape in (("w_gu", (2 * I, H)), ("w_dn", (H, I))):
-        x = torch.empty((E,) + shape, dtype=torch.bfloat16, device=device)
-        for e in range(E):
-            x[e] = synth.normal_bf16(shape, wl.seed, proj, e, std=0.02, device=device,
-                                     outlier_p=wl.outlier_p)
-        xs[proj] = x
-    outs = {p: nv.nvfp4_quantize(x) for p, x in xs.items()}
-    deq = {p: torch.empty_like(x) for p, x in xs.items()}
-    elts = sum(x.numel() for x in xs.values())
-
-    def q():
-        for p, x in xs.items():
-            nv.nvfp4_quantize(x, *outs[p])
-
-    def d():
-        for p in xs:
-            nv.nvfp4_dequantize(*outs[p], out=deq[p])
-
-    res = {}
-    for name, fn in (("quantize", q), ("dequantize", d)):
-        for _ in range(args.warmup):
-            fn()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.steps):
-            fn()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / args.steps
-        gbs = elts * 2.5625 / (ms / 1e3) / 1e9
-        res[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]}
-    qa = res["quantize"]["GB/s"]
-    roof = {"kernel": "quantize_kernel (amax + quantize, one cooperative launch)",
-            "bound": "hbm", "achieved": qa, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": qa / peaks["hbm_gbs"], "traffic": None,
-            "algorithmic_bytes": elts * 2.5625, "peak_source": peaks["source"] + " (burst copy)"}
-    return {"metric": "NVFP4 codec GB/s (whole layer)", "value": qa,
-            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": res["quantize"]["ms"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "elements": elts,
-                       "l2": "inputs (19.3 GB bf16) larger than L2"},
-            "roofline": roof, "codec": res,
-            "gpu_launches": 2 * args.steps}   # one quantize launch per projection per step
-
-
 # ----------------------------------------------------------------------------- reference arm
 REFERENCE_BUDGET_S = 150.0   # whole --impl reference run, warm-up included
 
 
 def run_reference(args):
-    """The CPU oracle as it stands, on the host cores, as the reference arm.  The unit of
-    work is one single-token decode step of the layer (8 of a pool of 16 experts; NVFP4
-    weights drawn directly as random codes and scales, since the oracle's cost does not
-    depend on values).  So that --steps K --warmup W ends within a few minutes, each step
-    runs a slice of the layer: the first i_rows of the I=2048 intermediate rows (gate, up
-    and the matching down columns), i_rows a multiple of 64 sized from a calibration run;
-    the oracle's work is linear in i_rows, and the rate is scaled to whole tokens."""
+    """The CPU oracle as it stands, on the host cores, as the reference arm, on the headline
+    workload (prefill, Zipf routing).  The unit of work is one token of that batch (routed to
+    8 of a pool of 16 experts; NVFP4 weights drawn directly as random codes and scales, since
+    the oracle's cost does not depend on values).  So that --steps K --warmup W ends within
+    a few minutes, each step runs a slice of one token's work: the first i_rows of the
+    I=2048 intermediate rows (gate, up and the matching down columns), i_rows a multiple of
+    64 sized from a calibration run; the oracle's work is linear in i_rows, and the rate is
+    scaled to whole tokens."""
     import oracle
+    wl = synth.PREFILL_T4096
     pool = 16
     n = args.steps + args.warmup
     x = synth.activations_bf16(n, H, 5)
-    ids, w = synth.routing(n, pool, K, seed=5)
+    ids, w = synth.routing(n, pool, K, seed=5, zipf_bias=wl.zipf_bias)
     # calibration (untimed): one step on a 64-row slice
     probe = random_nvfp4_pool(pool, i_rows=64)
     t0 = time.perf_counter()
@@ -448,13 +528,14 @@ def run_reference(args):
     sec = sum(times)
     frac = i_rows / I                   # fraction of a token's work per step
     v = len(times) * frac / sec
-    sample = (f"each step one single-token decode step (8 experts) on the first {i_rows} of "
-              f"{I} intermediate rows, i.e. {frac:.4f} of a token; rate scaled to whole tokens")
+    sample = (f"each step one token of the prefill batch (8 experts, Zipf routing) on the "
+              f"first {i_rows} of {I} intermediate rows, i.e. {frac:.4f} of a token; rate "
+              f"scaled to whole tokens")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sec / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": synth.DECODE_T1.name},
+            "config": {"workload": wl.name},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -480,15 +561,16 @@ def max_over_ranks(v, world, device):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=8192)
-    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode1")
+    ap.add_argument("--workload", default="all")
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--graph-steps", type=int, default=512)
     ap.add_argument("--e2e-steps", type=int, default=256)
-    ap.add_argument("--cpu-tokens", type=int, default=32)
+    ap.add_argument("--cpu-tokens", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-records", action="store_true")
     ap.add_argument("--experts", type=int, default=256,
                     help="experts in the layer (a smaller layer is only for profiling)")
     args = ap.parse_args()

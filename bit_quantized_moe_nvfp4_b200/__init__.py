@@ -22,7 +22,7 @@ __all__ = [
     "nvfp4_quantize", "nvfp4_quantize_workspace_size", "nvfp4_dequantize", "nvfp4_cast_f32",
     "moe_nvfp4_route", "moe_nvfp4_workspace_size", "moe_nvfp4_forward",
     "moe_nvfp4_read_error_flag", "moe_nvfp4_forward_profiled", "alloc_moe_workspace",
-    "moe_nvfp4_forward_static",
+    "moe_nvfp4_forward_static", "nvfp4_selftest_wait_timeout",
 ]
 
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "moe_nvfp4_route": (I32, [P, I64, I64, I64, P, P, P, P, P, P]),
         "moe_nvfp4_forward_static": (I32, [P, P, P, I64, I64, I64, I64, I64,
                                            P, P, P, P, P, P, P, P, P]),
+        "nvfp4_selftest_wait_timeout": (I32, [P, I32, I64, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -261,6 +262,17 @@ def moe_nvfp4_forward_static(x, topk_ids, topk_w, w_gu, s_gu, g_gu, w_dn, s_dn, 
         _ptr(g_gu), _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(out),
         _ptr(error_flag) if error_flag is not None else None, _stream(x.device)))
     return out
+
+
+def nvfp4_selftest_wait_timeout(flag: torch.Tensor, kind: int, limit_ns: int) -> None:
+    """Test hook: one kernel waits for something nothing completes (kind 0: an mbarrier
+    phase, 1: bulk-copy bytes, 2: a global counter) with a limit of limit_ns; the wait
+    runs out and bit 1 is ORed into flag's first int32 (device tensor, e.g. a forward
+    workspace)."""
+    if not isinstance(flag, torch.Tensor) or not flag.is_cuda:
+        raise ValueError("flag: expected a CUDA tensor")
+    _check(_lib().nvfp4_selftest_wait_timeout(_ptr(flag), int(kind), int(limit_ns),
+                                              _stream(flag.device)))
 
 
 def moe_nvfp4_read_error_flag(workspace: torch.Tensor) -> int:

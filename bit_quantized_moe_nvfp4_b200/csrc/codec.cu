@@ -73,27 +73,15 @@ __device__ __forceinline__ float global_scale_from_amax(uint32_t amax_bits) {
 // CTAs whose amax share of tensor t is merged.
 constexpr int kQwsHeader = 4;
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // Bounded wait (one thread) until *p >= want; a wait that gives up sets bit 1 of ws[0].
 __device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t want, uint32_t *ws,
                                            volatile int *abort) {
-  if (*abort) return false;
-  if (ld_acquire_gpu(p) >= want) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (ld_acquire_gpu(p) < want) {
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(ws, (uint32_t)kFlagWaitTimeout);
-      *abort = 1;
-      return false;
-    }
+  if (wait_geq(p, want, abort)) return true;
+  if (!*abort) {
+    atomicOr(ws, (uint32_t)kFlagWaitTimeout);
+    *abort = 1;
   }
-  return true;
+  return false;
 }
 
 // Quantize n tensors with one cooperative launch.  Warps 0-1 of every CTA take the amax of

@@ -27,6 +27,7 @@
 // rounded to f16.  bf16 has 8 significant bits and f16 11, so this is exact for every
 // element above 2^-31 * max|x_t| (smaller ones lose bits below f16's subnormal grid); the
 // dot products are rescaled by 2^-p_t in fp32.
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -1314,16 +1315,20 @@ __global__ void __launch_bounds__(32 * (CW + 1))
   }
 }
 
-int g_num_sms = 0;
-
+// SM count of the current device, looked up once per device (devices may differ).
 int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = kNumSMs;
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cached[kMaxDev];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDev) dev = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = kNumSMs;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return g_num_sms;
+  return n;
 }
 
 // Blocks of kernel k that fit on one SM at once with this block size and shared memory,
@@ -1384,7 +1389,7 @@ int launch_gateup_cfg(const MoeArgs &a, cudaStream_t s, int ctas_per_sm) {
   const uint32_t stage_bytes = (uint32_t)(2 * P * (a.H / 2) + 2 * span_bytes(P * (a.H / 16)));
   const int n = (int)(a.T * a.K);
   const Smem L = smem_layout(S, stage_bytes, CW, 2 * P * NT, n, (int)a.E, 0);
-  // the CTAs split the work evenly, so all of them must be resident at once
+  // one wave of resident CTAs that pull row chunks from a counter until none are left
   const int fit = resident_blocks(gemv_gateup_kernel<NT, P, S>, 32 * (CW + 2), L.total);
   if (fit <= 0) return fit < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
   return launch_pdl(gemv_gateup_kernel<NT, P, S>, dim3(num_sms() * min(ctas_per_sm, fit)),

@@ -15,9 +15,10 @@
 // kernel) have to be zero: they are zero when the library loads, and every call leaves them
 // zero.  Nothing else has to start at zero: the gate/up kernel writes every h row the down
 // kernel reads, the down kernel every y row the combine reads, and the flag is overwritten
-// by each call.  The array keeps the rows of the last call after it ends.  There is ONE array per device, shared by every call on that
-// device: calls on one stream are ordered and safe; calls that can overlap (different
-// streams or host threads on the same device) race on it.
+// by each call.  The array keeps the rows of the last call after it ends.  There is ONE
+// array per device, shared by every call on that device: calls on one stream are ordered
+// and safe; calls that can overlap (different streams or host threads on the same device)
+// race on it.
 #include <mutex>
 
 #include "moe.cuh"

@@ -70,11 +70,32 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 }
 
 // Wait for the phase with the given parity to complete; false if the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait_sleep(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait (one thread) until the global word *p reaches `want` (other CTAs add to it);
+// false if *abort was set or the limit ran out (the caller then records the timeout).
+__device__ __forceinline__ bool wait_geq(const uint32_t *p, uint32_t want, volatile int *abort,
+                                         uint64_t limit_ns = kWaitLimitNs) {
+  if (*abort) return false;
+  if (ld_acquire_gpu(p) >= want) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_gpu(p) < want) {
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
   return true;
 }

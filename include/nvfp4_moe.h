@@ -62,9 +62,9 @@ NVFP4_API const char *nvfp4_last_cuda_error(void);
 /* ---------------------------------------------------------------- codec */
 
 /* Bytes of workspace nvfp4_quantize needs: an error word, a per-tensor amax accumulator and
- * a per-tensor count of merged amax shares.  After the call, the first int32 of the workspace is 0, or
- * has bit 1 set if a device-side wait gave up (the outputs are then invalid); it can be read
- * with moe_nvfp4_read_error_flag. */
+ * a per-tensor count of merged amax shares.  After the call, the first int32 of the
+ * workspace is 0, or has bit 1 set if a device-side wait gave up (the outputs are then
+ * invalid); it can be read with moe_nvfp4_read_error_flag. */
 NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t n_tensors, int64_t rows, int64_t cols);
 
 /* Quantize n_tensors bf16 tensors of shape [rows, cols] to NVFP4 (page "GLM-5-NVFP4-MTP",
@@ -78,7 +78,7 @@ NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t n_tensors, int64_t rows, 
  * kept, so a small negative value gives 0x8); all codes 0 when d == 0.  Every step is an
  * IEEE fp32 operation rounded to nearest even, so results are reproducible bit for bit.
  * One cooperative kernel reads each tensor from HBM once: the quantize pass of a tensor
- * follows its amax pass while the tensor is still in L2. 
+ * follows its amax pass while the tensor is still in L2.
  * Requires cols % 32 == 0.  NaN/Inf inputs give unspecified codes.
  * Alignment: x 16 bytes, packed and global_scale 4 bytes, workspace 4 bytes.
  * Errors: EINVAL (null pointer, dimension <= 0, misaligned pointer), ESHAPE (cols % 32 != 0),
@@ -87,8 +87,10 @@ NVFP4_API int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t 
                    uint8_t *packed, uint8_t *scales, float *global_scale,
                    void *workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Dequantize NVFP4 to bf16: out = bf16( fp32(e2m1 * e4m3) * g ), the first product exact,
- * the multiply by g rounded once in fp32, then rounded to bf16 (nearest even).
+/* Dequantize NVFP4 to bf16 (page "GLM-5-NVFP4-MTP", "Model Description": each weight is a
+ * 4-bit value times the FP8 scale of its 16-element block, times the tensor's fp32 scale):
+ * out = bf16( fp32(e2m1 * e4m3) * g ), the first product exact, the multiply by g rounded
+ * once in fp32, then rounded to bf16 (nearest even).
  * Shapes as in nvfp4_quantize; requires cols % 32 == 0.  Alignment: packed and out 16
  * bytes, scales 2 bytes.  Errors: EINVAL (null or misaligned pointer), ESHAPE. */
 NVFP4_API int nvfp4_dequantize(const uint8_t *packed, const uint8_t *scales, const float *global_scale,
@@ -210,9 +212,10 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
  * Scratch: one array of NVFP4_STATIC_SCRATCH_BYTES per device, inside the library; no
  * call allocates or frees memory.  Only its first 8 bytes (the work counters of the
  * one-token kernels) must be zero at a call: they are zero when the library loads and every
- * call leaves them zero.  It keeps the last call's intermediate values after that call ends.  All calls on a device share it, so
- * calls that can overlap in time (different streams, or different host threads, on the
- * same device) race; calls on one stream are ordered and safe.  The first call on each
+ * call leaves them zero.  It keeps the last call's intermediate values after that call
+ * ends.  All calls on a device share it, so calls that can overlap in time (different
+ * streams, or different host threads, on the same device) race; calls on one stream are
+ * ordered and safe.  The first call on each
  * device looks the array's address up (cudaGetSymbolAddress): make that first call before
  * any stream capture begins on that device.
  * Errors: EINVAL (null or misaligned pointer, dimension <= 0), ESHAPE (the limits of
@@ -226,6 +229,24 @@ NVFP4_API int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *to
                                        const uint8_t *w_dn, const uint8_t *s_dn,
                                        const float *g_dn, __nv_bfloat16 *out,
                                        int32_t *error_flag, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- test hook */
+
+/* Runs the device-side failure path on purpose (the pages have no counterpart; this
+ * is test infrastructure for the library's bounded waits).  One kernel waits, with nothing
+ * to complete the wait, for
+ *   kind 0: an mbarrier phase that no thread arrives at;
+ *   kind 1: the bytes a barrier arrival announced, from a copy that is never issued;
+ *   kind 2: a global counter that no CTA advances,
+ * each bounded by limit_ns nanoseconds of %globaltimer instead of the kernels' 2 s.  When
+ * the limit runs out the kernel ORs bit 1 (NVFP4 "a device-side wait gave up") into *flag
+ * and returns; nothing faults and the CUDA context stays usable.  flag is a device int32
+ * (e.g. the first word of a forward workspace, so moe_nvfp4_read_error_flag reads it and the
+ * next forward on that workspace clears it), 4-byte aligned.
+ * Errors: EINVAL (null or misaligned flag, kind outside 0..2, limit_ns outside
+ * 1..1000000000), ECUDA. */
+NVFP4_API int nvfp4_selftest_wait_timeout(int32_t *flag, int kind, int64_t limit_ns,
+                                          cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -133,6 +133,20 @@ def test_route_argument_checks_run_before_cuda(lib):
     assert r(fake, 4, 2, 4096, fake, fake, fake, fake, None, None) == -2
 
 
+def test_selftest_argument_checks_run_before_cuda(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    f = lib.nvfp4_selftest_wait_timeout
+    f.restype = ctypes.c_int
+    f.argtypes = [P, ctypes.c_int, I64, P]
+    fake = ctypes.c_void_p(1 << 20)
+    assert f(None, 0, 1000000, None) == -1
+    assert f(ctypes.c_void_p((1 << 20) + 2), 0, 1000000, None) == -1   # misaligned
+    assert f(fake, 3, 1000000, None) == -1
+    assert f(fake, -1, 1000000, None) == -1
+    assert f(fake, 0, 0, None) == -1
+    assert f(fake, 0, 2000000000, None) == -1
+
+
 def test_oracle_and_product_share_no_code():
     """The product never imports, links or includes the oracle, and the oracle never
     imports or includes the product."""

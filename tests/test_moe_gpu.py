@@ -119,7 +119,9 @@ def test_single_token_edge_cases(nv, path):
 # ----------------------------------------------------------------------------- full size
 class FullLayer:
     """All 256 experts of the H=6144, I=2048 layer on the GPU, quantized by the GPU
-    quantizer (N(0, 0.02) bf16 weights)."""
+    quantizer (N(0, 0.02) bf16 weights).  The oracle's copy of an expert is quantized by
+    the oracle from the same seeded bf16 draw, after checking it equals the GPU bytes, and
+    kept per expert so that tokens sharing experts reuse it."""
 
     def __init__(self, nv, seed=0):
         wl = synth.DECODE_T1
@@ -134,25 +136,25 @@ class FullLayer:
             del x
         torch.cuda.empty_cache()
 
+    def _expert(self, e):
+        if e not in self._cache:
+            host = []
+            for pi, (proj, shape) in enumerate((("w_gu", (2 * self.I, self.H)),
+                                                ("w_dn", (self.H, self.I)))):
+                x = synth.normal_bf16(shape, self.seed, proj, e, std=0.02, device="cuda").cpu()
+                rp, rs, rg = oracle.quantize(x)
+                assert np.array_equal(self.dev[3 * pi][e].cpu().numpy(), rp[0])
+                assert np.array_equal(self.dev[3 * pi + 1][e].cpu().numpy(), rs[0])
+                assert np.array_equal(self.dev[3 * pi + 2][e:e + 1].cpu().numpy().view(np.uint32),
+                                      rg.view(np.uint32))
+                host += [rp[0], rs[0], rg[0]]
+            self._cache[e] = host
+        return self._cache[e]
+
     def oracle_inputs(self, experts):
-        """Oracle-quantized weights of the listed experts (after checking the GPU bytes)."""
-        key = tuple(experts)
-        if key in self._cache:
-            return self._cache[key]
-        host = []
-        for pi, (proj, shape) in enumerate((("w_gu", (2 * self.I, self.H)),
-                                            ("w_dn", (self.H, self.I)))):
-            x = torch.stack([synth.normal_bf16(shape, self.seed, proj, e, std=0.02,
-                                               device="cuda").cpu() for e in experts])
-            rp, rs, rg = oracle.quantize(x)
-            ix = torch.tensor(experts, device="cuda")
-            assert np.array_equal(self.dev[3 * pi][ix].cpu().numpy(), rp)
-            assert np.array_equal(self.dev[3 * pi + 1][ix].cpu().numpy(), rs)
-            assert np.array_equal(self.dev[3 * pi + 2][ix].cpu().numpy().view(np.uint32),
-                                  rg.view(np.uint32))
-            host += [rp, rs, rg]
-        self._cache = {key: host}
-        return host
+        """Oracle-quantized weights of the listed experts, stacked in that order."""
+        per = [self._expert(e) for e in experts]
+        return [np.stack([p[i] for p in per]) for i in range(6)]
 
 
 @pytest.fixture(scope="module")
@@ -161,25 +163,50 @@ def full(nv):
 
 
 def _check_sampled(full, x, ids, w, out, tokens):
-    for t in tokens:
-        experts = sorted(set(int(e) for e in ids[t]))
-        remap = {e: i for i, e in enumerate(experts)}
-        ids_t = torch.tensor([[remap[int(e)] for e in ids[t]]], dtype=torch.int32)
-        host = full.oracle_inputs(experts)
-        ref, ref64, bad = oracle.moe_forward(x[t:t + 1], ids_t, w[t:t + 1], *host)
-        assert bad == 0
-        compare_moe(out[t:t + 1], ref, ref64)
+    """Compare the listed tokens of `out` with the oracle, token by token, in one oracle call
+    over the union of their experts."""
+    tokens = sorted(set(int(t) for t in tokens))
+    experts = sorted(set(int(e) for t in tokens for e in ids[t]))
+    remap = {e: i for i, e in enumerate(experts)}
+    ids_s = torch.tensor([[remap[int(e)] for e in ids[t]] for t in tokens], dtype=torch.int32)
+    host = full.oracle_inputs(experts)
+    ref, ref64, bad = oracle.moe_forward(x[tokens], ids_s, w[tokens], *host)
+    assert bad == 0
+    for n, t in enumerate(tokens):
+        compare_moe(out[t:t + 1], ref[n:n + 1], ref64[n:n + 1])
+
+
+def prefill_probe_tokens(ids, tile_n, per_light=6, heavy=4):
+    """Tokens of a Zipf-routed batch whose outputs exercise the GEMM path's corner cases:
+    a token of each of the `per_light` lightest non-empty experts (a tile with only a few
+    occupied slots), the tokens of the first and last slot of the last partial n-tile of
+    each of the `heavy` heaviest experts, and one token from each half of the batch."""
+    a = ids.numpy()
+    T, K = a.shape
+    flat = a.reshape(-1)
+    counts = np.bincount(flat, minlength=int(flat.max()) + 1)
+    nonempty = np.nonzero(counts)[0]
+    chosen = []
+    for e in nonempty[np.argsort(counts[nonempty], kind="stable")[:per_light]]:
+        chosen.append(int(np.nonzero(flat == e)[0][0]) // K)
+    for e in np.argsort(-counts, kind="stable")[:heavy]:
+        pairs = np.nonzero(flat == e)[0]          # ascending pair index = slot order
+        n = pairs.size
+        first_of_last_tile = (n - 1) // tile_n * tile_n
+        chosen += [int(pairs[first_of_last_tile]) // K, int(pairs[-1]) // K]
+    chosen += [0, T // 2 + 1, T - 1]
+    return sorted(set(chosen))
 
 
 @pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
-@pytest.mark.parametrize("T", [1, 8, 64])
+@pytest.mark.parametrize("T", [1, 8, 32, 64])
 def test_full_layer_decode(nv, full, path, T):
     wl = synth.decode_batch(T)
     x = synth.activations_bf16(T, wl.H, 100 + T)
     ids, w = synth.routing(T, wl.E, wl.K, seed=100 + T)
     out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *full.dev, path=path)
     torch.cuda.synchronize()
-    _check_sampled(full, x, ids, w, out, tokens=[0, T - 1] if T > 1 else [0])
+    _check_sampled(full, x, ids, w, out, tokens=[0, T // 2, T - 1])
 
 
 def test_full_layer_single_token_calls_in_a_row(nv, full):
@@ -205,7 +232,10 @@ def test_full_layer_prefill(nv, full, path):
     ids, w = synth.routing(wl.T, wl.E, wl.K, seed=wl.seed, zipf_bias=wl.zipf_bias)
     out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *full.dev, path=path)
     torch.cuda.synchronize()
-    _check_sampled(full, x, ids, w, out, tokens=[0, 2049])
+    # n-tiles of 192 slots (the GEMM path's tile) and of 128 / 256 slots
+    tokens = sorted(set(sum((prefill_probe_tokens(ids, n) for n in (128, 192, 256)), [])))
+    assert len(tokens) >= 16
+    _check_sampled(full, x, ids, w, out, tokens=tokens)
     # the rest of the batch: cheap invariants over every token
     o = out.float()
     assert torch.isfinite(o).all()

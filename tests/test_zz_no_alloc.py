@@ -41,8 +41,9 @@ def _batch(T, E, K, H, seed):
     return x, ids.cuda(), w.cuda()
 
 
-@pytest.mark.parametrize("shape", [(32, 6144, 2048, 8, [16, 3]), (16, 192, 128, 4, [37, 5])],
-                         ids=["h6144_i2048", "h192_i128"])
+@pytest.mark.parametrize("shape", [(32, 6144, 2048, 8, [16, 3]), (16, 192, 128, 4, [37, 5]),
+                                   (32, 6144, 2048, 8, [1, 1, 1]), (16, 192, 128, 8, [1, 1])],
+                         ids=["h6144_i2048", "h192_i128", "h6144_i2048_t1", "h192_i128_t1"])
 def test_two_calls_match_workspace_forward(nv, shape):
     E, H, I, K, Ts = shape
     layer = _layer(nv, E, H, I, seed=11)
@@ -71,6 +72,30 @@ def test_bad_id_sets_flag(nv):
     ids[2, 1] = 0
     nv.moe_nvfp4_forward_static(x, ids, w, *layer, out=got, error_flag=flag)
     assert int(flag.item()) == 0
+
+
+def test_single_token_bad_id_then_clean_call(nv):
+    """One token runs the single-token kernels, which keep their work counters at the start
+    of the fixed scratch: a call with an out-of-range id raises the flag, and the clean calls
+    after it clear the flag and still match the workspace forward."""
+    E, H, I, K = 32, 6144, 2048, 8
+    layer = _layer(nv, E, H, I, seed=5)
+    flag = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    x, ids, w = _batch(1, E, K, H, seed=6)
+    ids_bad = ids.clone()
+    ids_bad[0, 3] = -2
+    got = nv.moe_nvfp4_forward_static(x, ids_bad, w, *layer, error_flag=flag)
+    ws = nv.alloc_moe_workspace(1, H, I, E, K)
+    ref = nv.moe_nvfp4_forward(x, ids_bad, w, *layer, workspace=ws, path=nv.PATH_GEMV)
+    _close(got, ref)
+    assert int(flag.item()) == nv.moe_nvfp4_read_error_flag(ws) == 1
+    for n in range(2):
+        x, ids, w = _batch(1, E, K, H, seed=7 + n)
+        got = nv.moe_nvfp4_forward_static(x, ids, w, *layer, error_flag=flag)
+        ref = nv.moe_nvfp4_forward(x, ids, w, *layer, workspace=ws, path=nv.PATH_GEMV)
+        torch.cuda.synchronize()
+        _close(got, ref)
+        assert int(flag.item()) == 0
 
 
 def test_batch_above_the_fixed_scratch_is_rejected(nv):
