@@ -27,9 +27,6 @@
 // rounded to f16.  bf16 has 8 significant bits and f16 11, so this is exact for every
 // element above 2^-31 * max|x_t| (smaller ones lose bits below f16's subnormal grid); the
 // dot products are rescaled by 2^-p_t in fp32.
-#include <atomic>
-#include <mutex>
-#include <vector>
 
 #include "moe.cuh"
 #include "pipeline.cuh"
@@ -149,20 +146,6 @@ __device__ __forceinline__ float dot16(uint32_t w0, uint32_t w1, const uint32_t 
   return a + b;
 }
 
-// Bulk copies move 16-byte-aligned runs of a multiple of 16 bytes.  A run of scale rows
-// (rows * cols/16 bytes) need not be aligned, so the aligned superset is copied instead:
-// it stays inside the expert's own scale block, whose size rows_total * cols/16 is a
-// multiple of 16 (rows and cols are multiples of 64).  Returns the bytes issued; the
-// wanted data starts `lead` = begin % 16 bytes into dst.
-__device__ __forceinline__ uint32_t bulk_g2s_span(void *dst, const uint8_t *block, int64_t begin,
-                                                  int64_t len, uint64_t *bar) {
-  const int64_t b = begin & ~int64_t(15);
-  const int64_t e = (begin + len + 15) & ~int64_t(15);
-  bulk_g2s(dst, block + b, (uint32_t)(e - b), bar);
-  return (uint32_t)(e - b);
-}
-
-__host__ __device__ __forceinline__ uint32_t span_bytes(int64_t len) { return (uint32_t)len + 32; }
 
 // ------------------------------------------------------------------ in-CTA routing
 // Shared-memory routing tables of one CTA.
@@ -1313,74 +1296,6 @@ __global__ void __launch_bounds__(32 * (CW + 1))
     }
     a.out[n0 + o] = __float2bfloat16_rn(acc);
   }
-}
-
-// SM count of the current device, looked up once per device (devices may differ).
-int num_sms() {
-  constexpr int kMaxDev = 64;
-  static std::atomic<int> cached[kMaxDev];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= kMaxDev) dev = 0;
-  int n = cached[dev].load(std::memory_order_relaxed);
-  if (n <= 0) {
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = kNumSMs;
-    cached[dev].store(n, std::memory_order_relaxed);
-  }
-  return n;
-}
-
-// Blocks of kernel k that fit on one SM at once with this block size and shared memory,
-// after raising the kernel's dynamic shared-memory limit to at least `smem`.  The limit is a
-// per-kernel, per-device attribute that only ever grows here (a call with less memory must
-// not lower it under a size another call still launches with), and the occupancy answer is
-// cached per kernel, device, block size and memory, so a steady stream of calls pays for
-// neither query again.
-template <typename Kern>
-int resident_blocks(Kern k, int threads, size_t smem) {
-  struct Limit {
-    const void *fn;
-    int dev;
-    size_t smem;
-  };
-  struct Entry {
-    const void *fn;
-    int dev, threads;
-    size_t smem;
-    int nb;
-  };
-  static std::mutex mu;
-  static std::vector<Limit> limits;
-  static std::vector<Entry> cache;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const void *fn = reinterpret_cast<const void *>(k);
-  std::lock_guard<std::mutex> lock(mu);
-  Limit *lim = nullptr;
-  for (Limit &l : limits)
-    if (l.fn == fn && l.dev == dev) lim = &l;
-  if (!lim || lim->smem < smem) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-      set_last_cuda_error(e);
-      return -1;
-    }
-    if (lim)
-      lim->smem = smem;
-    else
-      limits.push_back({fn, dev, smem});
-  }
-  for (const Entry &c : cache)
-    if (c.fn == fn && c.dev == dev && c.threads == threads && c.smem == smem) return c.nb;
-  int nb = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k, threads, smem);
-  if (e != cudaSuccess) {
-    set_last_cuda_error(e);
-    return -1;
-  }
-  if (cache.size() < 256) cache.push_back({fn, dev, threads, smem, nb});
-  return nb;
 }
 
 template <int NT, int P, int S>

@@ -56,6 +56,16 @@ int launch_gemm_gateup(const MoeArgs &a, cudaStream_t s);   // gather + gate/up 
 int launch_gemm_down(const MoeArgs &a, cudaStream_t s);
 int gemm_tile_n();
 
+// SM count of the current device, and blocks of kernel `fn` that fit on one SM with this
+// block size and dynamic shared memory (after raising the kernel's shared-memory limit to at
+// least `smem`); both cached per device.  resident_blocks returns -1 on a CUDA error.
+int num_sms();
+int resident_blocks_fn(const void *fn, int threads, size_t smem);
+template <typename Kern>
+int resident_blocks(Kern k, int threads, size_t smem) {
+  return resident_blocks_fn(reinterpret_cast<const void *>(k), threads, smem);
+}
+
 // Launch with programmatic dependent launch enabled (the kernel must call pdl_wait()
 // before it reads what the previous kernel wrote).
 template <typename Kern, typename... Args>

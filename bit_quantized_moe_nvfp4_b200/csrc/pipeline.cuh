@@ -110,6 +110,21 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// Bulk copies move 16-byte-aligned runs of a multiple of 16 bytes.  A run of scale rows
+// (rows * cols/16 bytes) need not be aligned, so the aligned superset is copied instead:
+// it stays inside the expert's own scale block, whose size rows_total * cols/16 is a
+// multiple of 16 (rows and cols are multiples of 64).  Returns the bytes issued; the
+// wanted data starts `lead` = begin % 16 bytes into dst.
+__device__ __forceinline__ uint32_t bulk_g2s_span(void *dst, const uint8_t *block, int64_t begin,
+                                                  int64_t len, uint64_t *bar) {
+  const int64_t b = begin & ~int64_t(15);
+  const int64_t e = (begin + len + 15) & ~int64_t(15);
+  bulk_g2s(dst, block + b, (uint32_t)(e - b), bar);
+  return (uint32_t)(e - b);
+}
+
+__host__ __device__ __forceinline__ uint32_t span_bytes(int64_t len) { return (uint32_t)len + 32; }
+
 // Named barrier among `threads` threads (a multiple of 32) with id 1..15.
 __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
