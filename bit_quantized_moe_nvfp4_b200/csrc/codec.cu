@@ -13,54 +13,23 @@
 namespace nvfp4 {
 
 // ------------------------------------------------------------------ quantize
-// The element codes without a division.  With q = RN(|x| / d) (IEEE division) the E2M1 code
-// counts the rounding thresholds q passes: q > 0.25, q >= 0.75, q > 1.25, q >= 1.75, q > 2.5,
-// q >= 3.5, q > 5 (a midpoint goes to the even code).  Each threshold m has an even fp32
-// significand, so  RN(a) > m  <=>  a > m + u/2  and  RN(a) >= m  <=>  a >= m - u'/2, with u
-// and u' the fp32 spacings just above and just below m.  For an fp32 |x| and a real bound t,
-// |x| > t <=> |x| > RD32(t) and |x| >= t <=> |x| >= RU32(t), and RD32((m + u/2) d) is one
-// fused multiply-add rounded down, fma_rd(m, d, (u/2) d), because (u/2) d is a power-of-two
-// scaling of d and so exact.  The seven fp32 thresholds of a block therefore give the same
-// codes as dividing every element by d.  (For d below 2^-100 the scaled term could lose bits
-// to underflow, and the bounds are formed in fp64 instead, where the products are exact.)
-struct Thresholds {
-  float t[7];   // t[0], t[2], t[4], t[6]: compare with >; t[1], t[3], t[5]: with >=
-};
-
-__device__ __forceinline__ Thresholds block_thresholds(float d) {
-  Thresholds r;
-  if (d >= 0x1p-100f) {
-    r.t[0] = __fmaf_rd(0.25f, d, __fmul_rn(d, 0x1p-26f));
-    r.t[1] = __fmaf_ru(0.75f, d, -__fmul_rn(d, 0x1p-25f));
-    r.t[2] = __fmaf_rd(1.25f, d, __fmul_rn(d, 0x1p-24f));
-    r.t[3] = __fmaf_ru(1.75f, d, -__fmul_rn(d, 0x1p-24f));
-    r.t[4] = __fmaf_rd(2.5f, d, __fmul_rn(d, 0x1p-23f));
-    r.t[5] = __fmaf_ru(3.5f, d, -__fmul_rn(d, 0x1p-23f));
-    r.t[6] = __fmaf_rd(5.0f, d, __fmul_rn(d, 0x1p-22f));
-  } else {
-    const double dd = (double)d;
-    r.t[0] = __double2float_rd((0.25 + 0x1p-26) * dd);
-    r.t[1] = __double2float_ru((0.75 - 0x1p-25) * dd);
-    r.t[2] = __double2float_rd((1.25 + 0x1p-24) * dd);
-    r.t[3] = __double2float_ru((1.75 - 0x1p-24) * dd);
-    r.t[4] = __double2float_rd((2.5 + 0x1p-23) * dd);
-    r.t[5] = __double2float_ru((3.5 - 0x1p-23) * dd);
-    r.t[6] = __double2float_rd((5.0 + 0x1p-22) * dd);
-  }
-  return r;
-}
-
-// E2M1 code of x for a block with divisor d > 0 (thresholds from block_thresholds(d)):
-// binary search over the seven thresholds, sign bit copied from x.
-__device__ __forceinline__ uint32_t e2m1_code(float x, const Thresholds &T) {
-  const float a = fabsf(x);
-  const bool b2 = a >= T.t[3];                         // code >= 4
-  const float t1 = b2 ? T.t[5] : T.t[1];               // code >= 6 / code >= 2
-  const bool b1 = a >= t1;
-  const float lo = b1 ? T.t[2] : T.t[0], hi = b1 ? T.t[6] : T.t[4];
-  const float t0 = b2 ? hi : lo;                       // the strict threshold above
-  const uint32_t c = (b2 ? 4u : 0u) + (b1 ? 2u : 0u) + (a > t0 ? 1u : 0u);
-  return c | ((__float_as_uint(x) >> 28) & 0x8u);
+// The element codes without a division per element.  The code of x is E2M1(q) with
+// q = RN(x / d), the IEEE quotient.  With r = RN(1/d), the product q' = RN(x * r) is within
+// 1.5 ulp of q (each of the two roundings is half an ulp, the reciprocal's error is carried
+// by the product once more), so q lies between q' * (1 - 2^-21) and q' * (1 + 2^-21), an
+// interval of +-4 ulp.  E2M1 rounding is monotone, so when the hardware convert
+// (round to nearest, ties to the even code, saturating, sign kept) gives the same code at
+// both ends, that is the code of q; only when a rounding midpoint of the E2M1 grid lies
+// inside the interval -- rare outside data placed on the midpoints -- is q formed by IEEE
+// division and converted.  The codes are therefore those of dividing every element by d.
+// (For d below 2^-100 the reciprocal could overflow, and every element is divided.)
+__device__ __forceinline__ uint32_t e2m1_pair_code(float x0, float x1, float d, float r) {
+  const float q0 = __fmul_rn(x0, r), q1 = __fmul_rn(x1, r);
+  constexpr float kBelow = 1.0f - 0x1p-21f, kAbove = 1.0f + 0x1p-21f;
+  const uint32_t lo = e2m1x2_rn_sat(__fmul_rn(q0, kBelow), __fmul_rn(q1, kBelow));
+  const uint32_t hi = e2m1x2_rn_sat(__fmul_rn(q0, kAbove), __fmul_rn(q1, kAbove));
+  if (lo == hi) return lo;
+  return e2m1x2_rn_sat(__fdiv_rn(x0, d), __fdiv_rn(x1, d));
 }
 
 // g = amax / 2688, IEEE division, 1 for an all-zero tensor.
@@ -109,10 +78,14 @@ __device__ __forceinline__ uint32_t quantize_half_block(uint4 v, float g, uint32
   const uint32_t sc = f32_to_e4m3(sv);
   const float d = __fmul_rn(e4m3_to_f32(sc), g);
   uint32_t word = 0;
-  if (d != 0.0f) {
-    const Thresholds T = block_thresholds(d);
+  if (d >= 0x1p-100f) {
+    const float r = __frcp_rn(d);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) word |= e2m1_code(f[k], T) << (4 * k);
+    for (int k = 0; k < 8; k += 2) word |= e2m1_pair_code(f[k], f[k + 1], d, r) << (4 * k);
+  } else if (d != 0.0f) {
+#pragma unroll
+    for (int k = 0; k < 8; k += 2)
+      word |= e2m1x2_rn_sat(__fdiv_rn(f[k], d), __fdiv_rn(f[k + 1], d)) << (4 * k);
   }
   *sc_out = sc;
   return word;

@@ -85,15 +85,19 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
   return (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
 }
 
-// fp32 -> E2M1 code by the rounding thresholds of the grid {0,.5,1,1.5,2,3,4,6}:
-// a midpoint goes to the neighbour with an even code (mantissa bit 0), anything at or
-// above 6 saturates, and the sign bit is copied from v (so -0.1 -> 0x8).
-__device__ __forceinline__ uint32_t f32_to_e2m1(float v) {
-  float a = fabsf(v);
-  uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-               (a >= 3.5f) + (a > 5.0f);
-  return c | ((__float_as_uint(v) >> 28) & 0x8u);
+// Two fp32 -> two E2M1 codes in one byte (lo in bits 0..3, hi in bits 4..7), by the
+// hardware convert: round to nearest, ties to the even code, saturating at +-6, sign kept
+// (so -0.1 -> 0x8).
+__device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\tcvt.u32.u8 %0, b;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
 }
+
+// fp32 -> E2M1 code (low nibble), rounded as e2m1x2_rn_sat rounds.
+__device__ __forceinline__ uint32_t f32_to_e2m1(float v) { return e2m1x2_rn_sat(v, 0.0f) & 0xFu; }
 
 // ------------------------------------------------------------------ memory
 __device__ __forceinline__ uint4 ldg_stream(const void *p) {

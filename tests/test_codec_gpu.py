@@ -53,6 +53,53 @@ def test_special_blocks(nv):
     _check_quant(nv, x)
 
 
+def _near_midpoint_tensor(rows, t_amax, rng):
+    """bf16 rows of 32 elements (two 16-element blocks) whose element quotients x / d lie on,
+    or within a few fp32 ulps of, an E2M1 rounding midpoint (0.25, 0.75, ..., 5), where the
+    search finds such values.  Element 0 fixes the tensor amax (hence g); element 0 of each
+    block fixes the block's d (computed with the oracle's own steps); the other 15 come from
+    an exhaustive search over the positive bf16 values, with random signs (random values
+    where the search finds nothing)."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    allv = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)   # positive bf16
+    g = np.float32(np.float32(t_amax) / np.float32(2688.0))
+    x = np.zeros((rows, 32), np.float32)
+    x[0, 0] = t_amax
+    for r in range(1, rows):
+        for blk in range(2):
+            b_amax = allv[rng.integers(0x3C00, 0x4400)]           # a block amax below t_amax
+            sv = np.float32(np.float32(b_amax / np.float32(6.0)) / g)
+            s8 = oracle.e4m3_encode(float(sv))
+            d = np.float32(np.float32(oracle.e4m3_value(s8)) * g)
+            with np.errstate(over="ignore", divide="ignore"):
+                q = (allv / d).astype(np.float32)
+            near = np.zeros(allv.shape, bool)
+            for m in mids:
+                near |= np.abs(q - m) <= 4 * np.spacing(m)
+            cand = allv[near & (allv <= b_amax)]
+            if cand.size == 0:
+                cand = allv[(allv <= b_amax) & (allv > b_amax / 64)]
+            sign = np.where(rng.random(15) < 0.5, -1.0, 1.0).astype(np.float32)
+            x[r, 16 * blk] = b_amax
+            x[r, 16 * blk + 1:16 * blk + 16] = rng.choice(cand, 15) * sign
+    return x
+
+
+def near_midpoint_input(rows=48, seed=17):
+    """Four tensors: global scales 1 and 0.75 (exact midpoint quotients: ties) and two
+    irregular ones (quotients next to a midpoint, where any exist)."""
+    rng = np.random.default_rng(seed)
+    ts = [_near_midpoint_tensor(rows, a, rng) for a in (2688.0, 2016.0, 1999.0, 2944.0)]
+    return torch.from_numpy(np.stack(ts)).to(torch.bfloat16)   # exact: all bf16 values
+
+
+def test_quantize_near_rounding_midpoints(nv):
+    """Element quotients on and next to every E2M1 rounding midpoint: the codes must be those
+    of dividing each element by its block's d (the quantizer's fast path defers to IEEE
+    division exactly there)."""
+    _check_quant(nv, near_midpoint_input())
+
+
 def test_dequantize_arbitrary_codes(nv):
     g = torch.Generator().manual_seed(3)
     packed = torch.randint(0, 256, (3, 20, 64), generator=g, dtype=torch.uint8)
