@@ -68,6 +68,10 @@ def _load():
             L.oracle_global_scale.argtypes = [P, I64]
             L.oracle_nvfp4_quantize.restype = None
             L.oracle_nvfp4_quantize.argtypes = [P, I64, I64, I64, P, P, P]
+            L.oracle_nvfp4_amax.restype = None
+            L.oracle_nvfp4_amax.argtypes = [P, I64, I64, P, ctypes.c_int]
+            L.oracle_nvfp4_quantize_with_amax.restype = None
+            L.oracle_nvfp4_quantize_with_amax.argtypes = [P, I64, I64, I64, P, P, P, P]
             L.oracle_nvfp4_dequantize.restype = None
             L.oracle_nvfp4_dequantize.argtypes = [P, P, P, I64, I64, I64, P]
             L.oracle_route.restype = I64
@@ -149,6 +153,40 @@ def quantize(x):
     scales = np.zeros((n, rows, cols // 16), np.uint8)
     g = np.zeros((n,), np.float32)
     _load().oracle_nvfp4_quantize(_p(xs), n, rows, cols, _p(packed), _p(scales), _p(g))
+    return packed, scales, g
+
+
+def amax(x, out=None, merge: bool = False):
+    """Per-tensor max |x| of bf16 [n, rows, cols] (or [rows, cols]) -> fp32 [n].  With
+    merge=True, `out` holds the amax of earlier calibration passes and becomes the
+    element-wise max of it and this pass's (page "GLM-5-NVFP4-MTP", "Calibration dataset")."""
+    xs = _u16(x)
+    if xs.ndim == 2:
+        xs = xs[None]
+    n = xs.shape[0]
+    per = xs.shape[1] * xs.shape[2]
+    if out is None:
+        out = np.zeros((n,), np.float32)
+    assert out.dtype == np.float32 and out.shape == (n,)
+    _load().oracle_nvfp4_amax(_p(xs), n, per, _p(out), int(bool(merge)))
+    return out
+
+
+def quantize_with_amax(x, amax_in):
+    """quantize() with the given per-tensor amax (e.g. a calibrated one) in place of each
+    tensor's own: g = amax / 2688 (1 for 0).  -> (packed, scales, g)."""
+    xs = _u16(x)
+    if xs.ndim == 2:
+        xs = xs[None]
+    n, rows, cols = xs.shape
+    assert cols % 16 == 0
+    am = _np(amax_in, np.float32).reshape(-1)
+    assert am.shape == (n,)
+    packed = np.zeros((n, rows, cols // 2), np.uint8)
+    scales = np.zeros((n, rows, cols // 16), np.uint8)
+    g = np.zeros((n,), np.float32)
+    _load().oracle_nvfp4_quantize_with_amax(_p(xs), n, rows, cols, _p(am), _p(packed),
+                                            _p(scales), _p(g))
     return packed, scales, g
 
 

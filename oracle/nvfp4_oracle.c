@@ -223,6 +223,56 @@ void oracle_nvfp4_quantize(const uint16_t *x, int64_t n_tensors, int64_t rows, i
     }
 }
 
+/* ------------------------------------------------------------------------------------- */
+/* Calibrated (static) global scales                                                     */
+/* ------------------------------------------------------------------------------------- */
+
+/* Per-tensor amax, max |x| over each tensor of `per` elements (exact: bf16 -> fp32).  Page
+ * "GLM-5-NVFP4-MTP", "Calibration dataset": several calibration passes are merged by
+ * element-wise max.  With merge == 0 amax[t] is set; with merge != 0 it becomes the larger
+ * of its value and this pass's, so calling once per pass leaves the merged amax. */
+void oracle_nvfp4_amax(const uint16_t *x, int64_t n_tensors, int64_t per, float *amax, int merge)
+{
+    for (int64_t t = 0; t < n_tensors; ++t) {
+        float a = 0.0f;
+        for (int64_t i = 0; i < per; ++i) {
+            float v = fabsf(oracle_bf16_to_f32(x[t * per + i]));
+            if (v > a)
+                a = v;
+        }
+        if (!merge || a > amax[t])
+            amax[t] = a;
+    }
+}
+
+/* Quantize with a given tensor amax (a calibrated one) in place of the tensor's own:
+ * g = amax_in / (6 * 448), 1 when amax_in == 0, then every block as in
+ * oracle_nvfp4_quantize.  Data beyond the calibrated range saturates: a block scale above
+ * 448 is stored as 448 and an element code above 6 as 6 (the E4M3 and E2M1 encoders
+ * saturate).  [Reading: amax_in >= 0 and finite; other values are not defined.] */
+void oracle_nvfp4_quantize_with_amax(const uint16_t *x, int64_t n_tensors, int64_t rows,
+                                     int64_t cols, const float *amax_in, uint8_t *packed,
+                                     uint8_t *scales, float *g_out)
+{
+    int64_t per = rows * cols;
+    for (int64_t t = 0; t < n_tensors; ++t) {
+        const uint16_t *xt = x + t * per;
+        float g = amax_in[t] == 0.0f ? 1.0f : amax_in[t] / (NVFP4_E2M1_MAX * NVFP4_E4M3_MAX);
+        g_out[t] = g;
+        #pragma omp parallel for schedule(static)
+        for (int64_t r = 0; r < rows; ++r) {
+            for (int64_t b = 0; b < cols / 16; ++b) {
+                uint8_t codes[16], sc;
+                quantize_block(xt + r * cols + b * 16, g, codes, &sc);
+                scales[t * rows * (cols / 16) + r * (cols / 16) + b] = sc;
+                uint8_t *dst = packed + t * rows * (cols / 2) + r * (cols / 2) + b * 8;
+                for (int j = 0; j < 8; ++j)
+                    dst[j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+            }
+        }
+    }
+}
+
 /* Dequantize: out = bf16( fp32( e2m1 * e4m3 ) * g ).  The first product is exact in fp32
  * (at most 6 significant bits); the multiply by g rounds once in fp32, and the conversion
  * to bf16 rounds a second time.  [Reading: the format sources give no dequantizer; this

@@ -284,3 +284,84 @@ def test_moe_special_cases():
     w2 = w[:, [1, 0]].contiguous()
     _, out64b, _ = oracle.moe_forward(x, ids2, w2, pg, sg, gg, pd, sd, gd)
     np.testing.assert_allclose(out64b, out64, rtol=1e-12, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- calibration
+def test_calibrated_hand_block():
+    """A hand-worked row quantized with a calibrated amax half the data's own: the block
+    scale and the codes saturate (tests/golden/calibrated_block.json gives the working)."""
+    gold = json.load(open(os.path.join(GOLDEN, "calibrated_block.json")))
+    x = torch.tensor(gold["x"], dtype=torch.float32).to(torch.bfloat16).view(1, 1, 32)
+    assert torch.equal(x.float().view(-1), torch.tensor(gold["x"]))
+    p, s, g = oracle.quantize_with_amax(x, np.array([gold["amax"]], np.float32))
+    assert float(g[0]) == gold["g"]
+    assert s.reshape(-1).tolist() == gold["scales"]
+    codes = np.stack([p.reshape(-1) & 15, p.reshape(-1) >> 4], axis=1).reshape(-1)
+    assert codes.tolist() == gold["codes"]
+    assert [f"{b:02x}" for b in p.reshape(-1)] == gold["packed_hex"]
+    deq = oracle.bf16_bits_to_f32(oracle.dequantize(p, s, g)).reshape(-1)
+    want = np.array(gold["dequant"], np.float32)
+    assert np.array_equal(deq, want) and np.array_equal(np.signbit(deq), np.signbit(want))
+
+
+def _planted(n, rows, cols, peaks, seed):
+    """bf16 tensors of values below 0.49 in magnitude, each with one planted maximum."""
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.rand((n, rows, cols), generator=g) * 0.98 - 0.49).to(torch.bfloat16)
+    for t, v in enumerate(peaks):
+        i = int(torch.randint(0, rows * cols, (1,), generator=g))
+        x.view(n, -1)[t, i] = v
+    return x
+
+
+def test_amax_is_the_planted_maximum():
+    peaks = [3.5, -7.25, 0.75, 1024.0]
+    x = _planted(4, 9, 48, peaks, 3)
+    assert oracle.amax(x).tolist() == [abs(v) for v in peaks]
+    assert oracle.amax(torch.zeros((2, 3, 16), dtype=torch.bfloat16)).tolist() == [0.0, 0.0]
+
+
+def test_amax_merge_is_elementwise_max_over_passes():
+    """Three calibration passes merged by element-wise max: the result is each tensor's
+    largest planted maximum, whatever the order of the passes; a running value larger than
+    a pass's amax is kept."""
+    passes = [[2.0, 9.0, 0.5], [9.0, -4.0, 0.75], [-4.0, 2.0, 0.625]]
+    xs = [_planted(3, 5, 32, p, 10 + i) for i, p in enumerate(passes)]
+    want = np.max(np.abs(np.array(passes)), axis=0).astype(np.float32)
+    for order in ([0, 1, 2], [2, 0, 1]):
+        acc = oracle.amax(xs[order[0]])
+        for i in order[1:]:
+            oracle.amax(xs[i], out=acc, merge=True)
+        assert acc.tolist() == want.tolist()
+    acc = np.array([100.0, 100.0, 100.0], np.float32)
+    assert oracle.amax(xs[0], out=acc, merge=True).tolist() == [100.0] * 3
+
+
+def test_quantize_with_own_amax_is_quantize():
+    """Given each tensor's own amax, the calibrated quantizer is the plain one."""
+    x = synth.normal_bf16((5, 12, 64), 23, "cal", std=0.02, outlier_p=0.02)
+    x[2] = 0.0
+    a, b = oracle.quantize_with_amax(x, oracle.amax(x)), oracle.quantize(x)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+@pytest.mark.parametrize("factor", [0.25, 4.0])
+def test_calibrated_range_invariants(factor):
+    """A calibrated amax below the data's saturates (scales at most 448, codes at most 6,
+    |dequantized| <= 6 * 448 * g); one above it leaves every block inside the E4M3 range."""
+    x = synth.normal_bf16((3, 16, 64), 29, "cal", std=1.0, outlier_p=0.01)
+    am = oracle.amax(x) * np.float32(factor)
+    p, s, g = oracle.quantize_with_amax(x, am)
+    assert np.array_equal(g, am / np.float32(2688.0))
+    assert int(s.max()) <= 0x7E
+    deq = oracle.bf16_bits_to_f32(oracle.dequantize(p, s, g)).astype(np.float64)
+    bound = 6.0 * 448.0 * g.astype(np.float64)[:, None, None]
+    assert np.all(np.abs(deq) <= bound * (1 + 2 ** -8))
+    if factor > 1:
+        assert int(s.max()) < 0x7E
+        xf = x.float().numpy().astype(np.float64)
+        # inside the range the dequantized block keeps the data's sign and the error is
+        # below one E2M1 step of the block
+        scl = np.repeat(np.vectorize(oracle.e4m3_value)(s), 16, axis=2) * g[:, None, None]
+        assert np.all(np.abs(deq - xf) <= scl * 2.0 + 1e-30)
