@@ -390,8 +390,28 @@ class Bench:
             for p in xs:
                 nv.nvfp4_dequantize(*outs[p], out=deq[p])
 
+        # calibrated scales: the amax pass, and the quantizer with the amax given
+        amx = {p: nv.nvfp4_amax(x) for p, x in xs.items()}
+
+        def am():
+            for p, x in xs.items():
+                nv.nvfp4_amax(x, out=amx[p])
+
+        def qa():
+            for p, x in xs.items():
+                nv.nvfp4_quantize_with_amax(x, amx[p], *outs[p])
+
+        def q2():   # amax pass, then the quantizer with that amax
+            am()
+            qa()
+
         res = {}
-        for name, fn in (("quantize", q), ("dequantize", d)):
+        legs = (("quantize", q, 2.5625, "quantize_kernel"),
+                ("dequantize", d, 2.5625, "dequantize_kernel"),
+                ("amax", am, 2.0, "amax_kernel"),
+                ("quantize_with_amax", qa, 2.5625, "quantize_amax_kernel"),
+                ("quantize_two_pass", q2, 2.5625, "amax_kernel + quantize_amax_kernel"))
+        for name, fn, bpe, kern in legs:
             for _ in range(warmup):
                 fn()
             torch.cuda.synchronize()
@@ -406,20 +426,19 @@ class Bench:
                 torch.cuda.synchronize()
             barrier(world)
             ms = max_over_ranks(e0.elapsed_time(e1), world, device) / steps
-            gbs = elts * 2.5625 / (ms / 1e3) / 1e9
-            kern = name + "_kernel"
+            gbs = elts * bpe / (ms / 1e3) / 1e9
             res[name] = {
                 "ms_per_layer": ms, "GB/s": gbs,
                 "roofline": {"kernel": kern, "bound": "hbm", "achieved": gbs,
                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": gbs / peaks["hbm_gbs"],
                              "traffic": measured_traffic(kern),
-                             "algorithmic_bytes": elts * 2.5625,
+                             "algorithmic_bytes": elts * bpe,
                              "peak_source": peaks["source"] + " (burst copy)"},
                 "clocks": clk.summary(),
-                # one launch per projection per layer
-                "gpu_launches": 2 * steps}
-        del xs, outs, deq, qws
+                # per projection per layer: one launch, two for the two-pass quantizer
+                "gpu_launches": (4 if name == "quantize_two_pass" else 2) * steps}
+        del xs, outs, deq, qws, amx
         torch.cuda.empty_cache()
         return {"metric": "NVFP4 codec GB/s (whole layer)", "unit": "GB/s",
                 "value": res["quantize"]["GB/s"], "steps": steps, "warmup": warmup,
@@ -428,7 +447,7 @@ class Bench:
                            "bytes_per_element": "2 (bf16) + 0.5625 (codes + scales)",
                            "l2": "inputs (19.3 GB bf16) larger than L2"},
                 "roofline": res["quantize"]["roofline"],
-                "quantize": res["quantize"], "dequantize": res["dequantize"]}
+                **res}
 
 
 SUB_DECODE_STEPS = {"decode1": 4096, "decode8": 1024, "decode32": 512, "decode64": 256}

@@ -22,7 +22,8 @@ __all__ = [
     "nvfp4_quantize", "nvfp4_quantize_workspace_size", "nvfp4_dequantize", "nvfp4_cast_f32",
     "moe_nvfp4_route", "moe_nvfp4_workspace_size", "moe_nvfp4_forward",
     "moe_nvfp4_read_error_flag", "moe_nvfp4_forward_profiled", "alloc_moe_workspace",
-    "moe_nvfp4_forward_static", "nvfp4_selftest_wait_timeout",
+    "moe_nvfp4_forward_static", "nvfp4_selftest_wait_timeout", "nvfp4_amax",
+    "nvfp4_quantize_with_amax",
 ]
 
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
@@ -61,6 +62,8 @@ def _load() -> ctypes.CDLL:
         "moe_nvfp4_forward_static": (I32, [P, P, P, I64, I64, I64, I64, I64,
                                            P, P, P, P, P, P, P, P, P]),
         "nvfp4_selftest_wait_timeout": (I32, [P, I32, I64, P]),
+        "nvfp4_amax": (I32, [P, I64, I64, I64, P, I32, P]),
+        "nvfp4_quantize_with_amax": (I32, [P, I64, I64, I64, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -134,6 +137,46 @@ def nvfp4_quantize(x: torch.Tensor, packed=None, scales=None, global_scale=None,
     _check(_lib().nvfp4_quantize(_ptr(x3), n, rows, cols, _ptr(packed), _ptr(scales),
                               _ptr(global_scale), _ptr(workspace), workspace.numel(),
                               _stream(dev)))
+    if squeeze:
+        return packed[0], scales[0], global_scale
+    return packed, scales, global_scale
+
+
+def nvfp4_amax(x: torch.Tensor, out=None, merge: bool = False) -> torch.Tensor:
+    """Per-tensor max |x| of bf16 [n, rows, cols] (or [rows, cols]) -> fp32 [n].  With
+    merge=True, `out` holds the amax of earlier calibration passes and becomes the
+    element-wise max of it and this pass's."""
+    _need(x, torch.bfloat16, "x")
+    x3 = x.unsqueeze(0) if x.dim() == 2 else x
+    n, rows, cols = x3.shape
+    if out is None:
+        if merge:
+            raise ValueError("merge=True needs the running amax in `out`")
+        out = torch.empty((n,), dtype=torch.float32, device=x.device)
+    _need(out, torch.float32, "out")
+    _check(_lib().nvfp4_amax(_ptr(x3), n, rows, cols, _ptr(out), int(bool(merge)),
+                             _stream(x.device)))
+    return out
+
+
+def nvfp4_quantize_with_amax(x: torch.Tensor, amax: torch.Tensor, packed=None, scales=None,
+                             global_scale=None):
+    """nvfp4_quantize with the per-tensor amax given (a calibrated one): g = amax / 2688.
+    -> (packed, scales, global_scale) as nvfp4_quantize."""
+    _need(x, torch.bfloat16, "x")
+    _need(amax, torch.float32, "amax")
+    squeeze = x.dim() == 2
+    x3 = x.unsqueeze(0) if squeeze else x
+    n, rows, cols = x3.shape
+    dev = x.device
+    if packed is None:
+        packed = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((n, rows, cols // 16), dtype=torch.uint8, device=dev)
+    if global_scale is None:
+        global_scale = torch.empty((n,), dtype=torch.float32, device=dev)
+    _check(_lib().nvfp4_quantize_with_amax(_ptr(x3), n, rows, cols, _ptr(amax), _ptr(packed),
+                                           _ptr(scales), _ptr(global_scale), _stream(dev)))
     if squeeze:
         return packed[0], scales[0], global_scale
     return packed, scales, global_scale

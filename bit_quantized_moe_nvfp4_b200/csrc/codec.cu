@@ -24,12 +24,65 @@ namespace nvfp4 {
 // division and converted.  The codes are therefore those of dividing every element by d.
 // (For d below 2^-100 the reciprocal could overflow, and every element is divided.)
 __device__ __forceinline__ uint32_t e2m1_pair_code(float x0, float x1, float d, float r) {
-  const float q0 = __fmul_rn(x0, r), q1 = __fmul_rn(x1, r);
+  const float2 q = __fmul2_rn(make_float2(x0, x1), make_float2(r, r));
   constexpr float kBelow = 1.0f - 0x1p-21f, kAbove = 1.0f + 0x1p-21f;
-  const uint32_t lo = e2m1x2_rn_sat(__fmul_rn(q0, kBelow), __fmul_rn(q1, kBelow));
-  const uint32_t hi = e2m1x2_rn_sat(__fmul_rn(q0, kAbove), __fmul_rn(q1, kAbove));
-  if (lo == hi) return lo;
+  const float2 lo = __fmul2_rn(q, make_float2(kBelow, kBelow));
+  const float2 hi = __fmul2_rn(q, make_float2(kAbove, kAbove));
+  const uint32_t a = e2m1x2_rn_sat(lo.x, lo.y), b = e2m1x2_rn_sat(hi.x, hi.y);
+  if (a == b) return a;
   return e2m1x2_rn_sat(__fdiv_rn(x0, d), __fdiv_rn(x1, d));
+}
+
+// The block scale code E4M3(RN(RN(amax_b / 6) / g)) the same way: with c = RN(1 / RN(6 g)),
+// RN(amax_b * c) is within 5 ulp of the twice-rounded quotient (five roundings of at most
+// half an ulp each), so when the E4M3 convert (nearest even, saturating) gives one code at
+// both ends of +-16 ulp around it, that is the code; otherwise the two divisions are taken.
+// `fast` is false for g below 2^-100, where c could overflow.
+__device__ __forceinline__ uint32_t block_scale_code(float amax_b, float g, float c, bool fast) {
+  if (fast) {
+    const float sp = __fmul_rn(amax_b, c);
+    const float2 e = __fmul2_rn(make_float2(sp, sp),
+                                make_float2(1.0f - 0x1p-20f, 1.0f + 0x1p-20f));
+    const uint32_t two = (uint32_t)__nv_cvt_float2_to_fp8x2(e, __NV_SATFINITE, __NV_E4M3);
+    if ((two & 0xFFu) == (two >> 8)) return two & 0xFFu;
+  }
+  return f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax_b, 6.0f), g));
+}
+
+// One 16-element block (two 16-byte words of bf16: element 2k in the low half of word k)
+// -> 8 bytes of codes (element 2j in the low nibble of byte j) and its scale code.
+__device__ __forceinline__ uint2 quantize_block16(const uint4 &v0, const uint4 &v1, float g,
+                                                  float c, bool fast, uint32_t *sc_out) {
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  uint32_t m = 0;   // max of |bf16| bit patterns (same order as the values)
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m = max(m, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+  const uint32_t sc = block_scale_code(__uint_as_float(m << 16), g, c, fast);
+  const float d = __fmul_rn(e4m3_to_f32(sc), g);
+  uint32_t out[2] = {0u, 0u};
+  if (d >= 0x1p-100f) {
+    const float r = __frcp_rn(d);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      out[k >> 2] |= e2m1_pair_code(bf16_lo(w[k]), bf16_hi(w[k]), d, r) << (8 * (k & 3));
+  } else if (d != 0.0f) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      out[k >> 2] |= e2m1x2_rn_sat(__fdiv_rn(bf16_lo(w[k]), d), __fdiv_rn(bf16_hi(w[k]), d))
+                     << (8 * (k & 3));
+  }
+  *sc_out = sc;
+  return make_uint2(out[0], out[1]);
+}
+
+// The per-tensor constants of quantize_block16: c = RN(1 / RN(6 g)), and whether the fast
+// scale path applies.
+struct BlockScaleConsts {
+  float c;
+  bool fast;
+};
+__device__ __forceinline__ BlockScaleConsts block_scale_consts(float g) {
+  return {__frcp_rn(__fmul_rn(6.0f, g)), g >= 0x1p-100f};
 }
 
 // g = amax / 2688, IEEE division, 1 for an all-zero tensor.
@@ -64,32 +117,6 @@ constexpr int kAmaxWarps = 2;
 constexpr int kAmaxThreads = 32 * kAmaxWarps;
 constexpr int kQuantThreads = 256 - kAmaxThreads;
 constexpr int kAmaxLoads = 16;   // 16-byte loads in flight per amax thread
-
-// One half block (8 elements) -> packed word; the block's scale code in *sc_out.  Lanes
-// 2i and 2i+1 hold the two halves of a block.
-__device__ __forceinline__ uint32_t quantize_half_block(uint4 v, float g, uint32_t *sc_out) {
-  const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                      bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-  float am = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) am = fmaxf(am, fabsf(f[k]));
-  am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-  const float sv = __fdiv_rn(__fdiv_rn(am, 6.0f), g);
-  const uint32_t sc = f32_to_e4m3(sv);
-  const float d = __fmul_rn(e4m3_to_f32(sc), g);
-  uint32_t word = 0;
-  if (d >= 0x1p-100f) {
-    const float r = __frcp_rn(d);
-#pragma unroll
-    for (int k = 0; k < 8; k += 2) word |= e2m1_pair_code(f[k], f[k + 1], d, r) << (4 * k);
-  } else if (d != 0.0f) {
-#pragma unroll
-    for (int k = 0; k < 8; k += 2)
-      word |= e2m1x2_rn_sat(__fdiv_rn(f[k], d), __fdiv_rn(f[k + 1], d)) << (4 * k);
-  }
-  *sc_out = sc;
-  return word;
-}
 
 // L2 eviction-priority policies for the two reads of a tensor: the amax pass marks lines to
 // be kept (the quantize pass comes back for them), the quantize pass marks them as last use.
@@ -177,38 +204,38 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     return;
   }
 
-  // ---- quantize: one thread per half block, four half blocks per thread per pass
+  // ---- quantize: one thread per 16-element block, two blocks per thread per pass
   const uint64_t last_use = l2_policy_evict_first();
   const int qt = threadIdx.x - kAmaxThreads;
   // the share boundaries are made even, so both halves of a block fall in one share
-  const int64_t q0 = v0 & ~int64_t(1);
-  const int64_t q1 = blockIdx.x + 1 == gridDim.x ? nvec : (v1 & ~int64_t(1));
+  const int64_t b0 = (v0 & ~int64_t(1)) / 2;
+  const int64_t b1 = blockIdx.x + 1 == gridDim.x ? nvec / 2 : (v1 & ~int64_t(1)) / 2;
   for (int t = 0; t < n_tensors; ++t) {
     if (qt == 0) wait_count(merged + t, gridDim.x, ws, abort);
     named_sync(2, kQuantThreads);
     const float g = global_scale_from_amax(__ldcg(amax_bits + t));
+    const BlockScaleConsts bc = block_scale_consts(g);
     if (blockIdx.x == 0 && qt == 0) global_scale[t] = g;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)t * per_tensor);
-    uint32_t *dst = reinterpret_cast<uint32_t *>(packed) + (int64_t)t * nvec;
+    uint2 *dst = reinterpret_cast<uint2 *>(packed) + (int64_t)t * (nvec / 2);
     uint8_t *sdst = scales + (int64_t)t * (nvec / 2);
-    // warp-uniform loop (the pair shuffle needs all lanes)
-    for (int64_t i0 = q0 + (qt & ~31); i0 < q1; i0 += 4 * kQuantThreads) {
-      uint4 v[4];
-      bool act[4];
+    for (int64_t i0 = b0 + qt; i0 < b1; i0 += 2 * kQuantThreads) {
+      uint4 v[2][2];
+      bool act[2];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int64_t i = i0 + k * kQuantThreads + lane;
-        act[k] = i < q1;
-        v[k] = act[k] ? ld_l2_hint(src + i, last_use) : make_uint4(0u, 0u, 0u, 0u);
+      for (int k = 0; k < 2; ++k) {
+        const int64_t b = i0 + k * kQuantThreads;
+        act[k] = b < b1;
+        v[k][0] = act[k] ? ld_l2_hint(src + 2 * b, last_use) : make_uint4(0u, 0u, 0u, 0u);
+        v[k][1] = act[k] ? ld_l2_hint(src + 2 * b + 1, last_use) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t sc;
-        const uint32_t word = quantize_half_block(v[k], g, &sc);
-        const int64_t i = i0 + k * kQuantThreads + lane;
+      for (int k = 0; k < 2; ++k) {
+        const int64_t b = i0 + k * kQuantThreads;
         if (act[k]) {
-          dst[i] = word;
-          if ((i & 1) == 0) sdst[i >> 1] = (uint8_t)sc;
+          uint32_t sc;
+          dst[b] = quantize_block16(v[k][0], v[k][1], g, bc.c, bc.fast, &sc);
+          sdst[b] = (uint8_t)sc;
         }
       }
     }
@@ -256,6 +283,103 @@ __global__ void __launch_bounds__(256) dequantize_kernel(
   }
 }
 
+// ------------------------------------------------------------------ calibrated scales
+// Page "GLM-5-NVFP4-MTP", "Calibration dataset": static scales from several calibration
+// passes, merged by element-wise max.  amax_kernel folds max |x| of each tensor into amax
+// (fp32 bits of a non-negative value order like the value, so an integer max merges them);
+// quantize_amax_kernel is the quantizer with that amax given, one read of the input.
+constexpr int kStreamLoads = 8;      // 16-byte loads in flight per thread (amax)
+constexpr int kQuantPerThread = 2;   // blocks per thread per pass (static quantizer)
+
+// CTA b takes the vectors [W b / G, W (b+1) / G) of all n tensors together (W vectors of 8
+// elements in all), tensor by tensor where its range crosses a boundary.
+__global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                   int64_t per_vec, int n_tensors,
+                                                   uint32_t *__restrict__ amax_bits) {
+  __shared__ uint32_t s_red[8];
+  const int64_t W = per_vec * n_tensors;
+  const int64_t v0 = W * blockIdx.x / gridDim.x, v1 = W * (blockIdx.x + 1) / gridDim.x;
+  const uint4 *src = reinterpret_cast<const uint4 *>(x);
+  for (int64_t seg = v0; seg < v1;) {
+    const int t = (int)(seg / per_vec);
+    const int64_t end = min(v1, (int64_t)(t + 1) * per_vec);
+    uint32_t m = 0;   // max of |bf16| bit patterns (same order as the values)
+    int64_t i = seg + threadIdx.x;
+    for (; i + (kStreamLoads - 1) * 256 < end; i += kStreamLoads * 256) {
+      uint4 v[kStreamLoads];
+#pragma unroll
+      for (int k = 0; k < kStreamLoads; ++k) v[k] = ldg_stream(src + i + k * 256);
+#pragma unroll
+      for (int k = 0; k < kStreamLoads; ++k) {
+        const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+      }
+    }
+    for (; i < end; i += 256) {
+      const uint4 v = ldg_stream(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < 8; ++w) m = max(m, s_red[w]);
+      if (m) atomicMax(amax_bits + t, m << 16);   // bf16 bits << 16 = fp32 bits
+    }
+    __syncthreads();
+    seg = end;
+  }
+}
+
+// One thread per 16-element block (32 bytes in, 8 bytes of codes and a scale byte out),
+// kQuantPerThread blocks per thread per pass.  g = amax / 2688 (1 for an amax of 0), IEEE
+// division.
+__global__ void __launch_bounds__(256) quantize_amax_kernel(
+    const __nv_bfloat16 *__restrict__ x, int64_t per_blk, int64_t n_blk,
+    const float *__restrict__ amax, uint8_t *__restrict__ packed,
+    uint8_t *__restrict__ scales, float *__restrict__ global_scale) {
+  const uint4 *src = reinterpret_cast<const uint4 *>(x);
+  uint2 *dst = reinterpret_cast<uint2 *>(packed);
+  const int64_t span = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x * kQuantPerThread + threadIdx.x;
+       i0 < n_blk; i0 += span * kQuantPerThread) {
+    uint4 v[kQuantPerThread][2];
+    bool act[kQuantPerThread];
+#pragma unroll
+    for (int k = 0; k < kQuantPerThread; ++k) {
+      const int64_t b = i0 + (int64_t)k * blockDim.x;
+      act[k] = b < n_blk;
+      v[k][0] = act[k] ? ldg_stream(src + 2 * b) : make_uint4(0u, 0u, 0u, 0u);
+      v[k][1] = act[k] ? ldg_stream(src + 2 * b + 1) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // the tensor of the thread's first block and its constants (a later block past the end
+    // of that tensor steps to the next one)
+    int t = (int)(i0 / per_blk);
+    float am = __ldg(amax + t);
+    float g = am == 0.0f ? 1.0f : __fdiv_rn(am, 2688.0f);
+    BlockScaleConsts bc = block_scale_consts(g);
+#pragma unroll
+    for (int k = 0; k < kQuantPerThread; ++k) {
+      const int64_t b = i0 + (int64_t)k * blockDim.x;
+      if (!act[k]) continue;
+      if (b >= (int64_t)(t + 1) * per_blk) {
+        while (b >= (int64_t)(t + 1) * per_blk) ++t;
+        am = __ldg(amax + t);
+        g = am == 0.0f ? 1.0f : __fdiv_rn(am, 2688.0f);
+        bc = block_scale_consts(g);
+      }
+      uint32_t sc;
+      dst[b] = quantize_block16(v[k][0], v[k][1], g, bc.c, bc.fast, &sc);
+      scales[b] = (uint8_t)sc;
+      if (b == (int64_t)t * per_blk) global_scale[t] = g;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ scalar casts
 __global__ void cast_kernel(const float *__restrict__ in, int64_t n, uint8_t *__restrict__ e4m3,
                             uint8_t *__restrict__ e2m1) {
@@ -290,8 +414,8 @@ extern "C" int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t
     return NVFP4_EINVAL;
   if (cols % 32 != 0) return NVFP4_ESHAPE;
   if (n_tensors >= (int64_t(1) << 24)) return NVFP4_ESHAPE;
-  // 16-byte loads of x, 4-byte stores of packed codes
-  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(packed) & 3) ||
+  // 16-byte loads of x, 8-byte stores of packed codes
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(packed) & 7) ||
       (reinterpret_cast<uintptr_t>(global_scale) & 3))
     return NVFP4_EINVAL;
   if (!workspace || ws_bytes < nvfp4_quantize_workspace_size(n_tensors, rows, cols) ||
@@ -355,5 +479,45 @@ extern "C" int nvfp4_cast_f32(const float *in, int64_t n, uint8_t *e4m3, uint8_t
                               cudaStream_t stream) {
   if (!in || n <= 0) return NVFP4_EINVAL;
   cast_kernel<<<grid_for(n, 256), 256, 0, stream>>>(in, n, e4m3, e2m1);
+  return check_launch();
+}
+
+extern "C" int nvfp4_amax(const __nv_bfloat16 *x, int64_t n_tensors, int64_t rows, int64_t cols,
+                          float *amax, int merge, cudaStream_t stream) {
+  if (!x || !amax || n_tensors <= 0 || rows <= 0 || cols <= 0) return NVFP4_EINVAL;
+  if (cols % 32 != 0 || n_tensors >= (int64_t(1) << 24)) return NVFP4_ESHAPE;
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(amax) & 3))
+    return NVFP4_EINVAL;
+  if (!merge) {
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * n_tensors, stream);
+    if (e != cudaSuccess) {
+      set_last_cuda_error(e);
+      return NVFP4_ECUDA;
+    }
+  }
+  const int64_t per_vec = rows * cols / 8;
+  const int64_t W = per_vec * n_tensors;
+  const int grid = (int)min((int64_t)kNumSMs * 8, max((int64_t)1, ceil_div(W, 256 * 32)));
+  amax_kernel<<<grid, 256, 0, stream>>>(x, per_vec, (int)n_tensors,
+                                        reinterpret_cast<uint32_t *>(amax));
+  return check_launch();
+}
+
+extern "C" int nvfp4_quantize_with_amax(const __nv_bfloat16 *x, int64_t n_tensors, int64_t rows,
+                                        int64_t cols, const float *amax, uint8_t *packed,
+                                        uint8_t *scales, float *global_scale,
+                                        cudaStream_t stream) {
+  if (!x || !amax || !packed || !scales || !global_scale || n_tensors <= 0 || rows <= 0 ||
+      cols <= 0)
+    return NVFP4_EINVAL;
+  if (cols % 32 != 0 || n_tensors >= (int64_t(1) << 24)) return NVFP4_ESHAPE;
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(packed) & 7) ||
+      (reinterpret_cast<uintptr_t>(amax) & 3) || (reinterpret_cast<uintptr_t>(global_scale) & 3))
+    return NVFP4_EINVAL;
+  const int64_t per_blk = rows * cols / 16;
+  const int64_t n_blk = per_blk * n_tensors;
+  const int grid = grid_for(ceil_div(n_blk, kQuantPerThread), 256);
+  quantize_amax_kernel<<<grid, 256, 0, stream>>>(x, per_blk, n_blk, amax, packed, scales,
+                                                 global_scale);
   return check_launch();
 }

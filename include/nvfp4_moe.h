@@ -80,7 +80,7 @@ NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t n_tensors, int64_t rows, 
  * One cooperative kernel reads each tensor from HBM once: the quantize pass of a tensor
  * follows its amax pass while the tensor is still in L2.
  * Requires cols % 32 == 0.  NaN/Inf inputs give unspecified codes.
- * Alignment: x 16 bytes, packed and global_scale 4 bytes, workspace 4 bytes.
+ * Alignment: x 16 bytes, packed 8 bytes, global_scale and workspace 4 bytes.
  * Errors: EINVAL (null pointer, dimension <= 0, misaligned pointer), ESHAPE (cols % 32 != 0),
  * EWORKSPACE (ws_bytes < nvfp4_quantize_workspace_size). */
 NVFP4_API int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t rows, int64_t cols,
@@ -96,6 +96,30 @@ NVFP4_API int nvfp4_quantize(const __nv_bfloat16 *x, int64_t n_tensors, int64_t 
 NVFP4_API int nvfp4_dequantize(const uint8_t *packed, const uint8_t *scales, const float *global_scale,
                      int64_t n_tensors, int64_t rows, int64_t cols, __nv_bfloat16 *out,
                      cudaStream_t stream);
+
+/* Calibrated (static) global scales (page "GLM-5-NVFP4-MTP", "Calibration dataset":
+ * several calibration passes, merged by element-wise max).
+ *
+ * nvfp4_amax: amax[t] = max |x| over tensor t of x [n_tensors, rows, cols] bf16 (exact).
+ * With merge == 0 amax is overwritten; with merge != 0 it becomes the element-wise max of
+ * its current value and this pass's, so one call per calibration pass on the same array
+ * leaves the merged amax.  amax: [n_tensors] fp32, device.  Requires cols % 32 == 0.
+ * Alignment: x 16 bytes, amax 4 bytes.  Errors: EINVAL, ESHAPE, ECUDA. */
+NVFP4_API int nvfp4_amax(const __nv_bfloat16 *x, int64_t n_tensors, int64_t rows, int64_t cols,
+                         float *amax, int merge, cudaStream_t stream);
+
+/* nvfp4_quantize with the tensor amax given (e.g. from nvfp4_amax over calibration data)
+ * instead of measured on x: g[t] = amax[t] / 2688 (1.0 for 0), written to global_scale,
+ * then every block exactly as nvfp4_quantize takes it.  Data beyond the calibrated range
+ * saturates (a block scale above 448 is stored as 448, an element above 6 * d as 6).
+ * One read of x; no workspace.  amax[t] must be finite and >= 0 (other values give
+ * unspecified codes).  Shapes, layout and alignment as nvfp4_quantize (x 16 bytes, packed
+ * 8 bytes, amax and global_scale 4 bytes).
+ * Errors: EINVAL, ESHAPE, ECUDA. */
+NVFP4_API int nvfp4_quantize_with_amax(const __nv_bfloat16 *x, int64_t n_tensors, int64_t rows,
+                                       int64_t cols, const float *amax, uint8_t *packed,
+                                       uint8_t *scales, float *global_scale,
+                                       cudaStream_t stream);
 
 /* Scalar format casts, element by element, exactly as the quantizer takes them:
  * e4m3[i] = E4M3(in[i]) and e2m1[i] = E2M1(in[i]) (nearest, ties to even, saturating,

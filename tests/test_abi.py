@@ -133,6 +133,23 @@ def test_route_argument_checks_run_before_cuda(lib):
     assert r(fake, 4, 2, 4096, fake, fake, fake, fake, None, None) == -2
 
 
+def test_calibration_argument_checks_run_before_cuda(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    a = lib.nvfp4_amax
+    a.restype = ctypes.c_int
+    a.argtypes = [P, I64, I64, I64, P, ctypes.c_int, P]
+    fake = ctypes.c_void_p(1 << 20)
+    assert a(None, 1, 16, 32, fake, 0, None) == -1
+    assert a(fake, 1, 16, 48, fake, 0, None) == -2
+    assert a(fake, 0, 16, 32, fake, 0, None) == -1
+    q = lib.nvfp4_quantize_with_amax
+    q.restype = ctypes.c_int
+    q.argtypes = [P, I64, I64, I64, P, P, P, P, P]
+    assert q(fake, 1, 16, 32, None, fake, fake, fake, None) == -1
+    assert q(fake, 1, 16, 40, fake, fake, fake, fake, None) == -2
+    assert q(ctypes.c_void_p((1 << 20) + 8), 1, 16, 32, fake, fake, fake, fake, None) == -1
+
+
 def test_selftest_argument_checks_run_before_cuda(lib):
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f = lib.nvfp4_selftest_wait_timeout
