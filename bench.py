@@ -22,9 +22,12 @@ sample, rank 0 at N=1), `e2e` (the same metric through the C ABI with pinned hos
 buffers, copies inside the timed region), `clocks`, `gpu_launches`.
 
 --impl reference times the CPU oracle itself on the host cores (the reference arm).
-With torchrun (N>1) every rank runs its own token stream (independent problems, weak
-scaling, no collective on the data path); only a barrier and a max-reduce of the times
-use NCCL.
+With torchrun (N>1) the layer runs expert parallel (--parallel ep, the default there):
+rank r holds only the experts e % N == r, every rank routes the same batch of T tokens,
+and one NCCL reduce-scatter sums the ranks' fp32 partial outputs (strong scaling: the job
+processes T tokens per step).  --parallel replicas instead runs an independent token stream
+per rank (weak scaling, no collective on the data path).  --parallel ep on one GPU runs the
+same code with one rank.
 """
 from __future__ import annotations
 
@@ -147,13 +150,15 @@ def physical_gpu(local_index: int) -> str:
 
 
 # ----------------------------------------------------------------------------- setup
-def build_layer(nv, device, seed=0):
-    """All 256 experts, bf16 N(0,0.02) drawn on the GPU and quantized by the library."""
+def build_layer(nv, device, seed=0, experts=None):
+    """The layer's experts (all E, or the listed global ids in that order), bf16 N(0,0.02)
+    drawn on the GPU per expert id and quantized by the library."""
+    experts = list(range(E)) if experts is None else list(experts)
     dev = []
     for proj, shape in (("w_gu", (2 * I, H)), ("w_dn", (H, I))):
-        x = torch.empty((E,) + shape, dtype=torch.bfloat16, device=device)
-        for e in range(E):
-            x[e] = synth.normal_bf16(shape, seed, proj, e, std=0.02, device=device)
+        x = torch.empty((len(experts),) + shape, dtype=torch.bfloat16, device=device)
+        for n, e in enumerate(experts):
+            x[n] = synth.normal_bf16(shape, seed, proj, e, std=0.02, device=device)
         dev += list(nv.nvfp4_quantize(x))
         del x
     torch.cuda.empty_cache()
@@ -364,6 +369,145 @@ class Bench:
         torch.cuda.empty_cache()
         return rec
 
+    def ep_record(self, name, steps, warmup):
+        """Expert parallelism over the `world` ranks: rank r holds only the experts
+        e % world == r; every rank routes the same batch, runs its experts
+        (moe_nvfp4_forward_ep), and an NCCL reduce-scatter sums the fp32 partials, leaving
+        each rank T/world rows of the layer output (bf16, moe_nvfp4_ep_reduce).  A step is
+        one batch of T tokens for the whole job (strong scaling)."""
+        from bit_quantized_moe_nvfp4_b200 import ep
+        nv, args, world, rank, device = self.nv, self.args, self.world, self.rank, self.device
+        peaks = self.peaks
+        wl = workload_of(name)
+        T = wl.T
+        mine = ep.local_experts(E, world, rank)
+        layer = build_layer(nv, device, experts=mine)
+        mode = "reduce_scatter" if T % world == 0 else "all_reduce"
+        moe = ep.ExpertParallelMoE(E, layer, mode=mode, path=args.path)
+        n_b = max(warmup, min(steps, 8))
+        # the same tokens on every rank: one seed for the whole job
+        xs, ids, ws_ = make_batches(wl, n_b, seed=1000, device=device)
+        stream = torch.cuda.current_stream(device)
+
+        def step(i):
+            return moe.forward(xs[i], ids[i], ws_[i])
+
+        for i in range(warmup):
+            step(i % n_b)
+        partial, summed, out, ws = moe._buffers(T, H, K, device)
+
+        def busy():
+            # this rank's experts only: the clock warm-up runs a different number of times
+            # on each rank, so it must not hold a collective
+            nv.moe_nvfp4_forward_ep(xs[0], ids[0], ws_[0], E, world, rank, *layer,
+                                    out=partial, workspace=ws, path=args.path)
+
+        barrier(world)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device(), stream, busy) as clk:
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for i in range(steps):
+                step(i % n_b)
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+        ms_step = ms_total / steps
+
+        # marked pass: this rank's experts, the exchange, the rounding
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        stage = {"experts": [], "exchange": [], "round": []}
+        for i in range(min(steps, n_b)):
+            marks[0].record(stream)
+            nv.moe_nvfp4_forward_ep(xs[i], ids[i], ws_[i], E, world, rank, *layer,
+                                    out=partial, workspace=ws, path=args.path)
+            marks[1].record(stream)
+            red = ep.reduce_partial(partial, mode=mode,
+                                    out=summed if mode == "reduce_scatter" else None)
+            marks[2].record(stream)
+            nv.moe_nvfp4_ep_reduce([red], out=out)
+            marks[3].record(stream)
+            torch.cuda.synchronize()
+            for j, k in enumerate(stage):
+                stage[k].append(marks[j].elapsed_time(marks[j + 1]))
+        stages = {k: statistics.mean(v) for k, v in stage.items()}
+        stages = {k: max_over_ranks(v, world, device) for k, v in stages.items()}
+
+        pairs = ids[:n_b].flatten().cpu()
+        local_pairs = float((pairs % world == rank).sum()) / n_b
+        fl_local = 2 * local_pairs * (3 * H * I)
+        achieved = fl_local / (stages["experts"] / 1e3) / 1e12
+        pk = peaks["bf16_tflops"]
+        exch_bytes = T * H * 4 * (world - 1) / world   # reduce-scatter bytes out of a rank
+        rec = {
+            "metric": METRIC, "value": T * steps / (ms_total / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "f16/bf16 products of NVFP4 weights, f32 accumulation",
+            "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) bf16 weights quantized to "
+                    "NVFP4)",
+            "config": {"workload": wl.name, "T": T, "H": H, "I": I, "E": E, "K": K,
+                       "parallelism": f"expert parallel over {world} GPU(s): experts "
+                                      f"e % {world} per rank, NCCL {mode} of fp32 partials",
+                       "weights": f"{len(mine)} experts per rank "
+                                  f"({len(mine) * EXPERT_BYTES / 1e9:.2f} GB)",
+                       "l2": "every step routes a batch over the rank's expert weights "
+                             "(>126 MB L2)",
+                       "timing": "stream launches (no graph), CUDA events, max over ranks"},
+            "stages_ms": stages,
+            "roofline": {"kernel": "this rank's experts (route + tcgen05 GEMMs + combine)",
+                         "bound": "tensor", "achieved": achieved, "peak": pk,
+                         "unit": "TFLOP/s", "frac": achieved / pk, "traffic": None,
+                         "algorithmic_flops": fl_local,
+                         "peak_source": peaks["source"] + " (cuBLAS bf16 burst)"},
+            "exchange": {"collective": f"NCCL {mode}", "bytes_out_per_rank": exch_bytes,
+                         "ms": stages["exchange"],
+                         "gbs": exch_bytes / (stages["exchange"] / 1e3) / 1e9
+                         if stages["exchange"] > 0 else None},
+            "gpu_launches": 6 * steps,   # route, gather, 2 GEMMs, combine, ep_reduce
+            "clocks": clk.summary(),
+        }
+        rec["e2e"] = self.ep_e2e(moe, wl, mode)
+        del moe, layer, xs, ids, ws_
+        torch.cuda.empty_cache()
+        return rec
+
+    def ep_e2e(self, moe, wl, mode):
+        """The expert-parallel step through the public API with host buffers: every rank
+        copies the batch in from pinned memory and its kept rows of the output back."""
+        from bit_quantized_moe_nvfp4_b200 import ep
+        device, world, rank = self.device, self.world, self.rank
+        T = wl.T
+        n = 4
+        xs = synth.activations_bf16(n * T, H, 77).view(n, T, H).pin_memory()
+        ids, w = synth.routing(n * T, E, K, seed=77, zipf_bias=wl.zipf_bias)
+        ids, w = ids.view(n, T, K).pin_memory(), w.view(n, T, K).pin_memory()
+        rows = ep.kept_rows(T, world, rank, mode)
+        out_h = torch.empty((n, rows.stop - rows.start, H), dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        idd = torch.empty((T, K), dtype=torch.int32, device=device)
+        wd = torch.empty((T, K), dtype=torch.float32, device=device)
+
+        def one(i):
+            xd.copy_(xs[i], non_blocking=True)
+            idd.copy_(ids[i], non_blocking=True)
+            wd.copy_(w[i], non_blocking=True)
+            out_h[i].copy_(moe.forward(xd, idd, wd), non_blocking=True)
+
+        one(0)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            one(i)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        return {"value": n * T / (ms / 1e3), "unit": "tokens/s", "steps": n,
+                "h2d_bytes_per_step": T * H * 2 + T * K * 4 * 2,
+                "d2h_bytes_per_step": (rows.stop - rows.start) * H * 2}
+
     def codec_record(self, steps, warmup):
         """Whole-layer quantize + dequantize of all 256 experts (gate/up and down)."""
         nv, world, device, peaks = self.nv, self.world, self.device, self.peaks
@@ -464,6 +608,8 @@ def run_ours(args, rank, world, device):
                     "gpu_launches": rec["quantize"]["gpu_launches"]})
         return rec
     main = "prefill" if args.workload == "all" else args.workload
+    if args.parallel == "ep":
+        return b.ep_record(main, args.steps, args.warmup)
     line = b.layer_record(main, args.steps, args.warmup, main=True)
     if args.workload == "all" and world == 1 and not args.no_sub_records:
         subs = []
@@ -590,6 +736,9 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub-records", action="store_true")
+    ap.add_argument("--parallel", choices=["ep", "replicas"], default=None,
+                    help="N>1: expert parallel (default) or independent replicas; "
+                         "ep also runs on one GPU (one rank)")
     ap.add_argument("--experts", type=int, default=256,
                     help="experts in the layer (a smaller layer is only for profiling)")
     args = ap.parse_args()
@@ -607,9 +756,15 @@ def main():
             print(json.dumps(run_reference(args)), flush=True)
         return
 
+    if args.parallel is None:
+        args.parallel = "ep" if world > 1 else "replicas"
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
+    if world > 1 or args.parallel == "ep":
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29511")
+        os.environ.setdefault("RANK", str(rank))
+        os.environ.setdefault("WORLD_SIZE", str(world))
         import datetime
         torch.distributed.init_process_group("nccl", device_id=device,
                                              timeout=datetime.timedelta(seconds=300))
@@ -618,7 +773,7 @@ def main():
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
-        if world > 1:
+        if torch.distributed.is_initialized():
             torch.distributed.destroy_process_group()
 
 

@@ -23,11 +23,13 @@ __all__ = [
     "moe_nvfp4_route", "moe_nvfp4_workspace_size", "moe_nvfp4_forward",
     "moe_nvfp4_read_error_flag", "moe_nvfp4_forward_profiled", "alloc_moe_workspace",
     "moe_nvfp4_forward_static", "nvfp4_selftest_wait_timeout", "nvfp4_amax",
-    "nvfp4_quantize_with_amax",
+    "nvfp4_quantize_with_amax", "moe_nvfp4_ep_local_experts", "moe_nvfp4_forward_ep",
+    "moe_nvfp4_ep_reduce", "EP_MAX_PARTS",
 ]
 
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
 WORKSPACE_ZERO_BYTES = 512   # head of a workspace that must be zero before first use
+EP_MAX_PARTS = 16            # partial outputs one moe_nvfp4_ep_reduce call sums
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libnvfp4moe.so")
 
@@ -64,6 +66,10 @@ def _load() -> ctypes.CDLL:
         "nvfp4_selftest_wait_timeout": (I32, [P, I32, I64, P]),
         "nvfp4_amax": (I32, [P, I64, I64, I64, P, I32, P]),
         "nvfp4_quantize_with_amax": (I32, [P, I64, I64, I64, P, P, P, P, P]),
+        "moe_nvfp4_ep_local_experts": (I64, [I64, I64, I64]),
+        "moe_nvfp4_forward_ep": (I32, [P, P, P, I64, I64, I64, I64, I64, I64, I64,
+                                       P, P, P, P, P, P, P, P, SZ, I32, P]),
+        "moe_nvfp4_ep_reduce": (I32, [P, I64, I64, I64, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -262,6 +268,65 @@ def moe_nvfp4_forward(x, topk_ids, topk_w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
         _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, I, E, K, _ptr(w_gu), _ptr(s_gu),
         _ptr(g_gu), _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(out), _ptr(workspace),
         workspace.numel(), int(path), _stream(x.device)))
+    return out
+
+
+def moe_nvfp4_ep_local_experts(E: int, ep_size: int, ep_rank: int) -> int:
+    """Experts rank ep_rank of ep_size owns (those e < E with e % ep_size == ep_rank)."""
+    return int(_lib().moe_nvfp4_ep_local_experts(E, ep_size, ep_rank))
+
+
+def moe_nvfp4_forward_ep(x, topk_ids, topk_w, E: int, ep_size: int, ep_rank: int,
+                         w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, out=None, workspace=None,
+                         path: int = PATH_AUTO) -> torch.Tensor:
+    """This rank's experts only (expert-parallel forward; see include/nvfp4_moe.h).
+
+    topk_ids hold global ids in [0, E); the weight tensors hold this rank's experts,
+    local index l = expert l * ep_size + ep_rank.  Returns the fp32 partial [T,H]."""
+    _need(x, torch.bfloat16, "x")
+    _need(topk_ids, torch.int32, "topk_ids")
+    _need(topk_w, torch.float32, "topk_w")
+    for t, n in ((w_gu, "w_gu"), (s_gu, "s_gu"), (w_dn, "w_dn"), (s_dn, "s_dn")):
+        _need(t, torch.uint8, n)
+    _need(g_gu, torch.float32, "g_gu")
+    _need(g_dn, torch.float32, "g_dn")
+    T, H = x.shape
+    K = topk_ids.shape[1]
+    E_loc, twoI, _ = w_gu.shape
+    if E_loc != moe_nvfp4_ep_local_experts(E, ep_size, ep_rank):
+        raise ValueError(f"w_gu holds {E_loc} experts; rank {ep_rank} of {ep_size} owns "
+                         f"{moe_nvfp4_ep_local_experts(E, ep_size, ep_rank)} of {E}")
+    I = twoI // 2
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    _need(out, torch.float32, "out")
+    if workspace is None:
+        workspace = alloc_moe_workspace(T, H, I, E_loc, K, x.device)
+    _check(_lib().moe_nvfp4_forward_ep(
+        _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, I, E, K, ep_size, ep_rank, _ptr(w_gu),
+        _ptr(s_gu), _ptr(g_gu), _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(out),
+        _ptr(workspace), workspace.numel(), int(path), _stream(x.device)))
+    return out
+
+
+def moe_nvfp4_ep_reduce(partials, out=None) -> torch.Tensor:
+    """bf16(partials[0] + partials[1] + ...) in fp32, in list order.  partials: fp32
+    [rows, cols] CUDA tensors (this device's, or peer memory it can read)."""
+    partials = list(partials)
+    if not partials:
+        raise ValueError("partials: at least one tensor")
+    for j, p in enumerate(partials):
+        _need(p, torch.float32, f"partials[{j}]")
+        if p.shape != partials[0].shape or p.dim() != 2:
+            raise ValueError("partials: fp32 tensors of one [rows, cols] shape")
+    rows, cols = partials[0].shape
+    dev = partials[0].device
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+    _need(out, torch.bfloat16, "out")
+    arr = (ctypes.c_void_p * len(partials))(*[p.data_ptr() for p in partials])
+    _check(_lib().moe_nvfp4_ep_reduce(arr, len(partials), rows, cols, _ptr(out),
+                                      _stream(dev)))
     return out
 
 

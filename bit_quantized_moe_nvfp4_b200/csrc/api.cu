@@ -103,23 +103,35 @@ static int record(cudaEvent_t const *ev, int i, cudaStream_t s) {
   return NVFP4_OK;
 }
 
+// Experts of rank `rank` of `size` under the e mod size partition (0 for bad arguments).
+static int64_t local_experts(int64_t E, int64_t size, int64_t rank) {
+  if (E <= 0 || size <= 0 || rank < 0 || rank >= size) return 0;
+  return (E - rank + size - 1) / size;
+}
+
+// One forward call.  E is the layer's expert count; `ep_size` > 1 runs the experts of rank
+// `ep_rank` only (the weight arrays then hold those experts) and writes the fp32 partial
+// out_f32 instead of out.
 static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w,
-                        int64_t T, int64_t H, int64_t I, int64_t E, int64_t K,
-                        const uint8_t *w_gu, const uint8_t *s_gu, const float *g_gu,
-                        const uint8_t *w_dn, const uint8_t *s_dn, const float *g_dn,
-                        __nv_bfloat16 *out, void *workspace, size_t ws_bytes, int path,
-                        cudaEvent_t const *ev, cudaStream_t stream) {
-  if (!x || !topk_ids || !topk_w || !w_gu || !s_gu || !g_gu || !w_dn || !s_dn || !g_dn || !out)
+                        int64_t T, int64_t H, int64_t I, int64_t E, int64_t K, int64_t ep_size,
+                        int64_t ep_rank, const uint8_t *w_gu, const uint8_t *s_gu,
+                        const float *g_gu, const uint8_t *w_dn, const uint8_t *s_dn,
+                        const float *g_dn, __nv_bfloat16 *out, float *out_f32, void *workspace,
+                        size_t ws_bytes, int path, cudaEvent_t const *ev, cudaStream_t stream) {
+  if (!x || !topk_ids || !topk_w || !w_gu || !s_gu || !g_gu || !w_dn || !s_dn || !g_dn ||
+      (!out && !out_f32))
     return NVFP4_EINVAL;
   if (T <= 0 || H <= 0 || I <= 0 || E <= 0 || K <= 0) return NVFP4_EINVAL;
+  if (ep_size < 1 || ep_rank < 0 || ep_rank >= ep_size || ep_size > E) return NVFP4_EINVAL;
   if (path != NVFP4_PATH_AUTO && path != NVFP4_PATH_GEMV && path != NVFP4_PATH_GEMM)
     return NVFP4_EINVAL;
   if (H % 64 || I % 64 || K > 16 || E > kMaxExperts || T * K >= (int64_t(1) << 31))
     return NVFP4_ESHAPE;
   if (!aligned16(x) || !aligned16(w_gu) || !aligned16(w_dn) || !aligned16(out) ||
-      !aligned16(s_gu) || !aligned16(s_dn))
+      !aligned16(out_f32) || !aligned16(s_gu) || !aligned16(s_dn))
     return NVFP4_EINVAL;
-  const WorkspaceLayout L = workspace_layout(T, H, I, E, K);
+  const int64_t E_loc = local_experts(E, ep_size, ep_rank);
+  const WorkspaceLayout L = workspace_layout(T, H, I, E_loc, K);
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return NVFP4_EWORKSPACE;
 
   char *ws = static_cast<char *>(workspace);
@@ -134,11 +146,13 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   a.s_dn = s_dn;
   a.g_dn = g_dn;
   a.out = out;
+  a.out_f32 = out_f32;
   a.T = T;
   a.H = H;
   a.I = I;
-  a.E = E;
+  a.E = E_loc;
   a.K = K;
+  a.map = ExpertMap{(int)E, (int)ep_size, (int)ep_rank};
   a.flag = reinterpret_cast<int32_t *>(ws + L.flag);
   a.work = reinterpret_cast<int32_t *>(ws + L.work);
   a.n_active = reinterpret_cast<int32_t *>(ws + L.n_active);
@@ -174,7 +188,8 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   RouteArgs r = {};
   r.ids = topk_ids;
   r.n_pairs = T * K;
-  r.E = (int)E;
+  r.E = (int)E_loc;
+  r.map = a.map;
   r.counts = a.counts;
   r.offsets = a.offsets;
   r.perm = a.perm;
@@ -202,8 +217,8 @@ extern "C" int moe_nvfp4_forward_path(const __nv_bfloat16 *x, const int32_t *top
                                       const uint8_t *w_dn, const uint8_t *s_dn,
                                       const float *g_dn, __nv_bfloat16 *out, void *workspace,
                                       size_t ws_bytes, int path, cudaStream_t stream) {
-  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
-                      out, workspace, ws_bytes, path, nullptr, stream);
+  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn,
+                      g_dn, out, nullptr, workspace, ws_bytes, path, nullptr, stream);
 }
 
 extern "C" int moe_nvfp4_forward_profiled(const __nv_bfloat16 *x, const int32_t *topk_ids,
@@ -217,8 +232,8 @@ extern "C" int moe_nvfp4_forward_profiled(const __nv_bfloat16 *x, const int32_t 
   if (!stage_events) return NVFP4_EINVAL;
   for (int i = 0; i < 5; ++i)
     if (!stage_events[i]) return NVFP4_EINVAL;
-  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
-                      out, workspace, ws_bytes, path,
+  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn,
+                      g_dn, out, nullptr, workspace, ws_bytes, path,
                       reinterpret_cast<cudaEvent_t const *>(stage_events), stream);
 }
 
@@ -230,6 +245,23 @@ extern "C" int moe_nvfp4_forward(const __nv_bfloat16 *x, const int32_t *topk_ids
                                  size_t ws_bytes, cudaStream_t stream) {
   return moe_nvfp4_forward_path(x, topk_ids, topk_w, T, H, I, E, K, w_gu, s_gu, g_gu, w_dn,
                                 s_dn, g_dn, out, workspace, ws_bytes, NVFP4_PATH_AUTO, stream);
+}
+
+extern "C" int64_t moe_nvfp4_ep_local_experts(int64_t E, int64_t ep_size, int64_t ep_rank) {
+  return local_experts(E, ep_size, ep_rank);
+}
+
+extern "C" int moe_nvfp4_forward_ep(const __nv_bfloat16 *x, const int32_t *topk_ids,
+                                    const float *topk_w, int64_t T, int64_t H, int64_t I,
+                                    int64_t E, int64_t K, int64_t ep_size, int64_t ep_rank,
+                                    const uint8_t *w_gu, const uint8_t *s_gu, const float *g_gu,
+                                    const uint8_t *w_dn, const uint8_t *s_dn, const float *g_dn,
+                                    float *out_partial, void *workspace, size_t ws_bytes,
+                                    int path, cudaStream_t stream) {
+  if (!out_partial) return NVFP4_EINVAL;
+  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, ep_size, ep_rank, w_gu, s_gu, g_gu,
+                      w_dn, s_dn, g_dn, nullptr, out_partial, workspace, ws_bytes, path,
+                      nullptr, stream);
 }
 
 extern "C" int moe_nvfp4_read_error_flag(const void *workspace, int32_t *host_flag,

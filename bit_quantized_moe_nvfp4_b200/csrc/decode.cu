@@ -156,23 +156,25 @@ struct CtaRoute {
   int *n_act;    // [1]
 };
 
-// All threads of the CTA: copy the ids, count pairs per expert (hist[E] is scratch), and
+// All threads of the CTA: copy the ids as local experts (kIdForeign / kIdBad for pairs
+// this device does not serve), count pairs per local expert (hist[E] is scratch), and
 // list the active experts with the exclusive prefix of their counts.  hist[e] ends up as
 // the active index of expert e (-1 if none).  Returns true if some id is out of range.
-__device__ bool cta_route(const int32_t *g_ids, int n, int E, CtaRoute r, int *hist) {
+__device__ bool cta_route(const int32_t *g_ids, int n, int E, ExpertMap map, CtaRoute r,
+                          int *hist) {
   __shared__ int s_bad;
   const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31;
   if (tid == 0) s_bad = 0;
   for (int e = tid; e < E; e += nth) hist[e] = 0;
   // ids are read past L1: they may have been written by the kernel this one follows
-  for (int p = tid; p < n; p += nth) r.ids[p] = __ldcg(g_ids + p);
+  for (int p = tid; p < n; p += nth) r.ids[p] = map.local(__ldcg(g_ids + p));
   __syncthreads();
   bool bad = false;
   for (int p = tid; p < n; p += nth) {
     const int v = r.ids[p];
-    if (v >= 0 && v < E)
+    if (v >= 0)
       atomicAdd(&hist[v], 1);
-    else
+    else if (v == kIdBad)
       bad = true;
   }
   if (bad) s_bad = 1;
@@ -240,16 +242,17 @@ __device__ int pairs_of_expert(const int *ids, int n, int e, int first, int lane
   return lane < NT ? mine : -1;
 }
 
-// Slot (row of h) of every pair: slot = first slot of its expert + stable rank; -1 for an
-// out-of-range id.  One warp; run[] is scratch of n_act ints.
-__device__ void warp_slots(const int *ids, int n, int E, const int *act_index, const int *act_off,
+// Slot (row of h) of every pair: slot = first slot of its expert + stable rank; -1 for a
+// pair this device does not serve.  ids are local (cta_route).  One warp; run[] is scratch
+// of n_act ints.
+__device__ void warp_slots(const int *ids, int n, const int *act_index, const int *act_off,
                            int n_act, int *run, int *slot, int lane) {
   for (int a = lane; a < n_act; a += 32) run[a] = act_off[a];
   __syncwarp();
   for (int base = 0; base < n; base += 32) {
     const int p = base + lane;
-    const int v = p < n ? ids[p] : -1;
-    const bool valid = v >= 0 && v < E;
+    const int v = p < n ? ids[p] : kIdBad;
+    const bool valid = v >= 0;
     const unsigned key = valid ? (unsigned)v : 0x80000000u | (unsigned)lane;
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
     const int rank = __popc(peers & ((1u << lane) - 1u));
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumerWarps + 2), NT == 1 ? 2 : 1)
 #pragma unroll
     for (int i = 0; i < 4; ++i) xv[i] = __ldcg(xp + i);
   }
-  const bool bad = cta_route(a.ids, n, E, R, hist);
+  const bool bad = cta_route(a.ids, n, E, a.map, R, hist);
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.flag) *a.flag = bad ? kFlagBadId : 0;
   pdl_launch_dependents();  // the down kernel may start routing and prefetching
 
@@ -806,7 +809,7 @@ __global__ void __launch_bounds__(32 * (kGuWarps + 1 + kGuFinal), 1)
   if (MODE == 0) pdl_wait();   // x and the ids come from earlier kernels
   // (MODE 1: the ids were complete before the gate/up kernel let this grid start, so the
   // routing and the weight stream start before griddepcontrol.wait)
-  const bool bad = cta_route(a.ids, n, E, R, hist);
+  const bool bad = cta_route(a.ids, n, E, a.map, R, hist);
   if (MODE == 0 && blockIdx.x == 0 && threadIdx.x == 0 && a.flag) *a.flag = bad ? kFlagBadId : 0;
   float *wts = reinterpret_cast<float *>(smem + L.wts);
   if (MODE == 1) {   // the pair weights, read once here instead of once per tile and output
@@ -1120,9 +1123,9 @@ __global__ void __launch_bounds__(32 * (CW + 1))
   }
   // The ids were complete before the gate/up kernel let this grid start; reading them
   // (and the weights) before griddepcontrol.wait overlaps this prologue with its tail.
-  cta_route(a.ids, n, E, R, hist);
+  cta_route(a.ids, n, E, a.map, R, hist);
   const int n_act = *R.n_act;
-  if (warp == 1) warp_slots(R.ids, n, E, hist, R.act_off, n_act, run, slot_of, lane);
+  if (warp == 1) warp_slots(R.ids, n, hist, R.act_off, n_act, run, slot_of, lane);
   __syncthreads();
 
   const int n0 = blockIdx.x * nb;
@@ -1294,7 +1297,10 @@ __global__ void __launch_bounds__(32 * (CW + 1))
       const int sl = slot_of[k];
       if (sl >= 0) acc += yk[(size_t)sl * nb + o] * __ldg(a.w + k);
     }
-    a.out[n0 + o] = __float2bfloat16_rn(acc);
+    if (a.out_f32)
+      a.out_f32[n0 + o] = acc;
+    else
+      a.out[n0 + o] = __float2bfloat16_rn(acc);
   }
 }
 

@@ -18,7 +18,10 @@ struct MoeArgs {
   const uint8_t *s_dn;        // [E, H, I/16]
   const float *g_dn;          // [E]
   __nv_bfloat16 *out;         // [T, H]
-  int64_t T, H, I, E, K;
+  float *out_f32;             // [T, H] fp32 partial output instead of out (expert parallel),
+                              //   or null
+  int64_t T, H, I, E, K;      // E: experts on this device (the length of the weight arrays)
+  ExpertMap map;              // routed (global) id -> local expert
   // workspace
   int32_t *flag;              // [1] error bits
   int32_t *work;              // [2] work counters of the one-token gate/up kernel (zero)

@@ -109,6 +109,7 @@ extern "C" int moe_nvfp4_forward_static(const __nv_bfloat16 *x, const int32_t *t
   a.I = I;
   a.E = E;
   a.K = K;
+  a.map = whole_layer(E);
   a.flag = error_flag;   // may be NULL: the kernels then skip the flag writes
   a.work = reinterpret_cast<int32_t *>(base);
   a.h = reinterpret_cast<__nv_bfloat16 *>(base + kStaticHead);

@@ -32,10 +32,10 @@ __global__ void __launch_bounds__(1024) route_kernel(RouteArgs a) {
   // 1. histogram
   int bad = 0;
   for (int64_t p = tid; p < n; p += blockDim.x) {
-    int id = a.ids[p];
-    if (id >= 0 && id < E)
+    const int id = a.map.local(a.ids[p]);
+    if (id >= 0)
       atomicAdd(&cnt[id], 1);
-    else
+    else if (id == kIdBad)
       bad = 1;
   }
   if (bad) atomicOr(&s_bad, 1);
@@ -105,8 +105,8 @@ __global__ void __launch_bounds__(1024) route_kernel(RouteArgs a) {
     for (int i = tid; i < 32 * E; i += blockDim.x) wpos[i] = 0;
     __syncthreads();
     const int64_t p = c0 + tid;
-    const int id = p < n ? a.ids[p] : -1;
-    const bool valid = id >= 0 && id < E;
+    const int id = p < n ? a.map.local(a.ids[p]) : kIdBad;
+    const bool valid = id >= 0;
     // invalid pairs get a key no valid id can match, unique per lane
     const unsigned key = valid ? (unsigned)id : 0x80000000u | (unsigned)lane;
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
@@ -183,6 +183,7 @@ extern "C" int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, in
   a.ids = topk_ids;
   a.n_pairs = T * K;
   a.E = (int)E;
+  a.map = whole_layer(E);
   a.counts = counts;
   a.offsets = offsets;
   a.perm = perm;

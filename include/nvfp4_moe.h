@@ -216,6 +216,57 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
                     int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
                     int32_t *error_flag, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- expert parallelism */
+
+/* Page "GLM-5-NVFP4-MTP", "How to Run", serves the model across several GPUs.  The routed
+ * experts shard by expert: rank r of G ("ep_size") owns the experts e in [0, E) with
+ * e mod G == r and stores expert e at local index e / G.  Every rank runs
+ * moe_nvfp4_forward_ep on the same tokens and routing; the layer output is
+ * bf16(sum over ranks of their fp32 partials), which moe_nvfp4_ep_reduce forms (over
+ * peer-mapped partials, or as the rounding step after a library reduction of them). */
+#define NVFP4_EP_MAX_PARTS 16
+
+/* Number of experts rank ep_rank owns: ceil((E - ep_rank) / ep_size); 0 for E <= 0,
+ * ep_size <= 0 or ep_rank outside [0, ep_size). */
+NVFP4_API int64_t moe_nvfp4_ep_local_experts(int64_t E, int64_t ep_size, int64_t ep_rank);
+
+/* The forward of rank ep_rank's experts only.  Arguments as moe_nvfp4_forward_path, except:
+ *   E            the layer's expert count; topk_ids hold ids in [0, E)
+ *   ep_size      ranks sharing the experts, 1 <= ep_size <= E
+ *   ep_rank      this rank, 0 <= ep_rank < ep_size
+ *   w_gu .. g_dn this rank's experts, local index l = expert l * ep_size + ep_rank:
+ *                [E_loc, ...] with E_loc = moe_nvfp4_ep_local_experts(E, ep_size, ep_rank)
+ *   out_partial  [T, H] fp32, 16-byte aligned: for every token the sum, over its slots k
+ *                in ascending order whose expert this rank owns, of topk_w[t,k] * y(t,k),
+ *                with y as in moe_nvfp4_forward; 0 for a token with none.
+ * Slots routed to another rank's expert are skipped without error; ids outside [0, E) are
+ * skipped and set bit 0 of the workspace error flag, as in moe_nvfp4_forward.  Workspace:
+ * moe_nvfp4_workspace_size(T, H, I, E_loc, K) bytes (the size for E covers it).
+ * With ep_size 1 the call computes moe_nvfp4_forward's sum before its bf16 rounding.
+ * Errors: EINVAL (also ep_size / ep_rank out of range, null out_partial), ESHAPE,
+ * EWORKSPACE, ECUDA. */
+NVFP4_API int moe_nvfp4_forward_ep(const __nv_bfloat16 *x, const int32_t *topk_ids,
+                                   const float *topk_w, int64_t T, int64_t H, int64_t I,
+                                   int64_t E, int64_t K, int64_t ep_size, int64_t ep_rank,
+                                   const uint8_t *w_gu, const uint8_t *s_gu, const float *g_gu,
+                                   const uint8_t *w_dn, const uint8_t *s_dn, const float *g_dn,
+                                   float *out_partial, void *workspace, size_t ws_bytes,
+                                   int path, cudaStream_t stream);
+
+/* out = bf16_RN(partials[0] + partials[1] + ... + partials[n_parts-1]), elementwise, in
+ * fp32 and in that order (deterministic whichever rank finished first).
+ *   partials  HOST array of n_parts device pointers, each [rows, cols] fp32 row-major,
+ *             16-byte aligned; a pointer may be another GPU's memory that this device can
+ *             read (peer access enabled, or an IPC / virtual-memory mapping)
+ *   out       [rows, cols] bf16, 8-byte aligned, on this device; must not overlap a partial
+ * Limits: 1 <= n_parts <= NVFP4_EP_MAX_PARTS, cols % 4 == 0.  rows == 0 enqueues nothing.
+ * The caller orders the call after every partial is complete (an event or a barrier across
+ * ranks) and keeps the partials unchanged until it has run.
+ * Errors: EINVAL (null or misaligned pointer, n_parts <= 0, rows < 0, cols <= 0), ESHAPE,
+ * ECUDA. */
+NVFP4_API int moe_nvfp4_ep_reduce(const float *const *partials, int64_t n_parts, int64_t rows,
+                                  int64_t cols, __nv_bfloat16 *out, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- fixed-scratch forward */
 
 /* Bytes of the fixed scratch of moe_nvfp4_forward_static: it holds 256 bytes of counters,
@@ -239,9 +290,9 @@ NVFP4_API int moe_nvfp4_route(const int32_t *topk_ids, int64_t T, int64_t K, int
  * call leaves them zero.  It keeps the last call's intermediate values after that call
  * ends.  All calls on a device share it, so calls that can overlap in time (different
  * streams, or different host threads, on the same device) race; calls on one stream are
- * ordered and safe.  The first call on each
- * device looks the array's address up (cudaGetSymbolAddress): make that first call before
- * any stream capture begins on that device.
+ * ordered and safe.  The first call on each device looks the array's address up
+ * (cudaGetSymbolAddress): make that first call before any stream capture begins on that
+ * device.
  * Errors: EINVAL (null or misaligned pointer, dimension <= 0), ESHAPE (the limits of
  * moe_nvfp4_forward, a batch whose h and y do not fit NVFP4_STATIC_SCRATCH_BYTES, or a
  * shape the GEMV path does not take: T*K > 1024, H > 6144, I > 6144, or I > 3072 with

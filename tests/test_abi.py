@@ -150,6 +150,47 @@ def test_calibration_argument_checks_run_before_cuda(lib):
     assert q(ctypes.c_void_p((1 << 20) + 8), 1, 16, 32, fake, fake, fake, fake, None) == -1
 
 
+def test_expert_parallel_argument_checks_run_before_cuda(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    f = lib.moe_nvfp4_forward_ep
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, I64, I64, I64, I64, I64, I64, I64, P, P, P, P, P, P, P, P,
+                  ctypes.c_size_t, ctypes.c_int, P]
+    fake = ctypes.c_void_p(1 << 20)
+    good = dict(T=1, H=6144, I=2048, E=256, K=8, G=8, r=3)
+
+    def call(ptr=fake, out=fake, ws=fake, ws_bytes=1 << 40, **over):
+        d = dict(good, **over)
+        return f(ptr, ptr, ptr, d["T"], d["H"], d["I"], d["E"], d["K"], d["G"], d["r"],
+                 ptr, ptr, ptr, ptr, ptr, ptr, out, ws, ws_bytes, 0, None)
+
+    assert call(out=None) == -1
+    assert call(G=0) == -1
+    assert call(r=8) == -1
+    assert call(r=-1) == -1
+    assert call(G=300) == -1                 # more ranks than experts
+    assert call(out=ctypes.c_void_p((1 << 20) + 4)) == -1   # partial not 16-byte aligned
+    assert call(H=6100) == -2
+    assert call(ws_bytes=16) == -3
+    n = lib.moe_nvfp4_ep_local_experts
+    n.restype = I64
+    n.argtypes = [I64, I64, I64]
+    assert [n(10, 4, r) for r in range(4)] == [3, 3, 2, 2]
+    assert n(10, 4, 4) == 0 and n(0, 1, 0) == 0
+    red = lib.moe_nvfp4_ep_reduce
+    red.restype = ctypes.c_int
+    red.argtypes = [P, I64, I64, I64, P, P]
+    ptrs = (ctypes.c_void_p * 17)(*([1 << 20] * 17))
+    assert red(None, 1, 4, 8, fake, None) == -1
+    assert red(ptrs, 0, 4, 8, fake, None) == -1
+    assert red(ptrs, 17, 4, 8, fake, None) == -2
+    assert red(ptrs, 2, 4, 6, fake, None) == -2
+    assert red(ptrs, 2, 4, 8, None, None) == -1
+    bad = (ctypes.c_void_p * 2)(1 << 20, (1 << 20) + 8)
+    assert red(bad, 2, 4, 8, fake, None) == -1          # a partial not 16-byte aligned
+    assert red(ptrs, 2, 0, 8, fake, None) == 0          # no rows: nothing to enqueue
+
+
 def test_selftest_argument_checks_run_before_cuda(lib):
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f = lib.nvfp4_selftest_wait_timeout

@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import synth
-from helpers import Layer, compare_moe
+from helpers import Layer, check_sampled, compare_moe, prefill_probe_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -117,85 +117,9 @@ def test_single_token_edge_cases(nv, path):
 
 
 # ----------------------------------------------------------------------------- full size
-class FullLayer:
-    """All 256 experts of the H=6144, I=2048 layer on the GPU, quantized by the GPU
-    quantizer (N(0, 0.02) bf16 weights).  The oracle's copy of an expert is quantized by
-    the oracle from the same seeded bf16 draw, after checking it equals the GPU bytes, and
-    kept per expert so that tokens sharing experts reuse it."""
-
-    def __init__(self, nv, seed=0):
-        wl = synth.DECODE_T1
-        self.E, self.H, self.I, self.seed = wl.E, wl.H, wl.I, seed
-        self._cache = {}
-        self.dev = []
-        for proj, shape in (("w_gu", (2 * self.I, self.H)), ("w_dn", (self.H, self.I))):
-            x = torch.empty((self.E,) + shape, dtype=torch.bfloat16, device="cuda")
-            for e in range(self.E):
-                x[e] = synth.normal_bf16(shape, seed, proj, e, std=0.02, device="cuda")
-            self.dev += list(nv.nvfp4_quantize(x))
-            del x
-        torch.cuda.empty_cache()
-
-    def _expert(self, e):
-        if e not in self._cache:
-            host = []
-            for pi, (proj, shape) in enumerate((("w_gu", (2 * self.I, self.H)),
-                                                ("w_dn", (self.H, self.I)))):
-                x = synth.normal_bf16(shape, self.seed, proj, e, std=0.02, device="cuda").cpu()
-                rp, rs, rg = oracle.quantize(x)
-                assert np.array_equal(self.dev[3 * pi][e].cpu().numpy(), rp[0])
-                assert np.array_equal(self.dev[3 * pi + 1][e].cpu().numpy(), rs[0])
-                assert np.array_equal(self.dev[3 * pi + 2][e:e + 1].cpu().numpy().view(np.uint32),
-                                      rg.view(np.uint32))
-                host += [rp[0], rs[0], rg[0]]
-            self._cache[e] = host
-        return self._cache[e]
-
-    def oracle_inputs(self, experts):
-        """Oracle-quantized weights of the listed experts, stacked in that order."""
-        per = [self._expert(e) for e in experts]
-        return [np.stack([p[i] for p in per]) for i in range(6)]
-
-
 @pytest.fixture(scope="module")
-def full(nv):
-    return FullLayer(nv)
-
-
-def _check_sampled(full, x, ids, w, out, tokens):
-    """Compare the listed tokens of `out` with the oracle, token by token, in one oracle call
-    over the union of their experts."""
-    tokens = sorted(set(int(t) for t in tokens))
-    experts = sorted(set(int(e) for t in tokens for e in ids[t]))
-    remap = {e: i for i, e in enumerate(experts)}
-    ids_s = torch.tensor([[remap[int(e)] for e in ids[t]] for t in tokens], dtype=torch.int32)
-    host = full.oracle_inputs(experts)
-    ref, ref64, bad = oracle.moe_forward(x[tokens], ids_s, w[tokens], *host)
-    assert bad == 0
-    for n, t in enumerate(tokens):
-        compare_moe(out[t:t + 1], ref[n:n + 1], ref64[n:n + 1])
-
-
-def prefill_probe_tokens(ids, tile_n, per_light=6, heavy=4):
-    """Tokens of a Zipf-routed batch whose outputs exercise the GEMM path's corner cases:
-    a token of each of the `per_light` lightest non-empty experts (a tile with only a few
-    occupied slots), the tokens of the first and last slot of the last partial n-tile of
-    each of the `heavy` heaviest experts, and one token from each half of the batch."""
-    a = ids.numpy()
-    T, K = a.shape
-    flat = a.reshape(-1)
-    counts = np.bincount(flat, minlength=int(flat.max()) + 1)
-    nonempty = np.nonzero(counts)[0]
-    chosen = []
-    for e in nonempty[np.argsort(counts[nonempty], kind="stable")[:per_light]]:
-        chosen.append(int(np.nonzero(flat == e)[0][0]) // K)
-    for e in np.argsort(-counts, kind="stable")[:heavy]:
-        pairs = np.nonzero(flat == e)[0]          # ascending pair index = slot order
-        n = pairs.size
-        first_of_last_tile = (n - 1) // tile_n * tile_n
-        chosen += [int(pairs[first_of_last_tile]) // K, int(pairs[-1]) // K]
-    chosen += [0, T // 2 + 1, T - 1]
-    return sorted(set(chosen))
+def full(full_layer):
+    return full_layer
 
 
 @pytest.mark.parametrize("path", PATHS, ids=["gemv", "gemm"])
@@ -206,7 +130,7 @@ def test_full_layer_decode(nv, full, path, T):
     ids, w = synth.routing(T, wl.E, wl.K, seed=100 + T)
     out = nv.moe_nvfp4_forward(x.cuda(), ids.cuda(), w.cuda(), *full.dev, path=path)
     torch.cuda.synchronize()
-    _check_sampled(full, x, ids, w, out, tokens=[0, T // 2, T - 1])
+    check_sampled(full, x, ids, w, out, tokens=[0, T // 2, T - 1])
 
 
 def test_full_layer_single_token_calls_in_a_row(nv, full):
@@ -222,7 +146,7 @@ def test_full_layer_single_token_calls_in_a_row(nv, full):
                                    path=1)
         torch.cuda.synchronize()
         assert torch.all(ws[:nv.WORKSPACE_ZERO_BYTES].view(torch.int32)[1:] == 0)
-        _check_sampled(full, x, ids, w, out, tokens=[0])
+        check_sampled(full, x, ids, w, out, tokens=[0])
 
 
 @pytest.mark.parametrize("path", [2, 0], ids=["gemm", "auto"])
@@ -235,7 +159,7 @@ def test_full_layer_prefill(nv, full, path):
     # n-tiles of 192 slots (the GEMM path's tile) and of 128 / 256 slots
     tokens = sorted(set(sum((prefill_probe_tokens(ids, n) for n in (128, 192, 256)), [])))
     assert len(tokens) >= 16
-    _check_sampled(full, x, ids, w, out, tokens=tokens)
+    check_sampled(full, x, ids, w, out, tokens=tokens)
     # the rest of the batch: cheap invariants over every token
     o = out.float()
     assert torch.isfinite(o).all()
