@@ -24,7 +24,8 @@ __all__ = [
     "moe_nvfp4_read_error_flag", "moe_nvfp4_forward_profiled", "alloc_moe_workspace",
     "moe_nvfp4_forward_static", "nvfp4_selftest_wait_timeout", "nvfp4_amax",
     "nvfp4_quantize_with_amax", "moe_nvfp4_ep_local_experts", "moe_nvfp4_forward_ep",
-    "moe_nvfp4_ep_reduce", "EP_MAX_PARTS",
+    "moe_nvfp4_ep_reduce", "EP_MAX_PARTS", "moe_nvfp4_router", "moe_nvfp4_forward_logits",
+    "moe_nvfp4_shared_expert", "moe_nvfp4_layer", "moe_nvfp4_layer_workspace_size",
 ]
 
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
@@ -70,6 +71,14 @@ def _load() -> ctypes.CDLL:
         "moe_nvfp4_forward_ep": (I32, [P, P, P, I64, I64, I64, I64, I64, I64, I64,
                                        P, P, P, P, P, P, P, P, SZ, I32, P]),
         "moe_nvfp4_ep_reduce": (I32, [P, I64, I64, I64, P, P]),
+        "moe_nvfp4_router": (I32, [P, I64, I64, I64, P, P, P]),
+        "moe_nvfp4_shared_workspace_size": (SZ, [I64, I64]),
+        "moe_nvfp4_shared_expert": (I32, [P, I64, I64, I64, P, P, P, P, P, SZ, P]),
+        "moe_nvfp4_layer_workspace_size": (SZ, [I64, I64, I64, I64, I64, I64]),
+        "moe_nvfp4_layer": (I32, [P, P, I64, I64, I64, I64, I64, P, P, P, P, P, P, P, P, I64,
+                                  P, P, P, P, SZ, I32, P]),
+        "moe_nvfp4_forward_logits": (I32, [P, P, I64, I64, I64, I64, I64,
+                                           P, P, P, P, P, P, P, P, P, P, SZ, I32, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -268,6 +277,107 @@ def moe_nvfp4_forward(x, topk_ids, topk_w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
         _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, I, E, K, _ptr(w_gu), _ptr(s_gu),
         _ptr(g_gu), _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(out), _ptr(workspace),
         workspace.numel(), int(path), _stream(x.device)))
+    return out
+
+
+def moe_nvfp4_router(logits: torch.Tensor, K: int, ids=None, w=None):
+    """Top-K experts and renormalised softmax weights from fp32 logits [T, E] (see
+    include/nvfp4_moe.h).  Returns (ids int32 [T, K], w fp32 [T, K])."""
+    _need(logits, torch.float32, "logits")
+    T, E = logits.shape
+    if ids is None:
+        ids = torch.empty((T, K), dtype=torch.int32, device=logits.device)
+    if w is None:
+        w = torch.empty((T, K), dtype=torch.float32, device=logits.device)
+    _need(ids, torch.int32, "ids")
+    _need(w, torch.float32, "w")
+    _check(_lib().moe_nvfp4_router(_ptr(logits), T, E, K, _ptr(ids), _ptr(w),
+                                   _stream(logits.device)))
+    return ids, w
+
+
+def moe_nvfp4_forward_logits(x, router_logits, K: int, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
+                             out=None, ids_out=None, w_out=None, workspace=None,
+                             path: int = PATH_AUTO) -> torch.Tensor:
+    """The router on fp32 logits [T, E], then the layer on its decisions, in one call.
+    ids_out / w_out (optional, [T, K]) receive the router's decisions."""
+    _need(x, torch.bfloat16, "x")
+    _need(router_logits, torch.float32, "router_logits")
+    for t, n in ((w_gu, "w_gu"), (s_gu, "s_gu"), (w_dn, "w_dn"), (s_dn, "s_dn")):
+        _need(t, torch.uint8, n)
+    _need(g_gu, torch.float32, "g_gu")
+    _need(g_dn, torch.float32, "g_dn")
+    if ids_out is not None:
+        _need(ids_out, torch.int32, "ids_out")
+    if w_out is not None:
+        _need(w_out, torch.float32, "w_out")
+    T, H = x.shape
+    E, twoI, _ = w_gu.shape
+    I = twoI // 2
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = alloc_moe_workspace(T, H, I, E, K, x.device)
+    _check(_lib().moe_nvfp4_forward_logits(
+        _ptr(x), _ptr(router_logits), T, H, I, E, K, _ptr(w_gu), _ptr(s_gu), _ptr(g_gu),
+        _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(out), _ptr(ids_out), _ptr(w_out),
+        _ptr(workspace), workspace.numel(), int(path), _stream(x.device)))
+    return out
+
+
+def moe_nvfp4_shared_expert(x, w_gu, w_dn, routed=None, out=None, workspace=None):
+    """The BF16 shared expert (see include/nvfp4_moe.h): out = bf16(routed + W_dn .
+    bf16(silu(W_g x) * W_u x)) per token.  x bf16 [T,H]; w_gu bf16 [2Is,H]; w_dn bf16
+    [H,Is]; routed fp32 [T,H] or None.  Returns out bf16 [T,H]."""
+    _need(x, torch.bfloat16, "x")
+    _need(w_gu, torch.bfloat16, "w_gu")
+    _need(w_dn, torch.bfloat16, "w_dn")
+    if routed is not None:
+        _need(routed, torch.float32, "routed")
+    T, H = x.shape
+    Is = w_gu.shape[0] // 2
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        n = int(_lib().moe_nvfp4_shared_workspace_size(T, Is))
+        workspace = torch.empty((max(n, 16),), dtype=torch.uint8, device=x.device)
+    _check(_lib().moe_nvfp4_shared_expert(_ptr(x), T, H, Is, _ptr(w_gu), _ptr(w_dn),
+                                          _ptr(routed), _ptr(out), _ptr(workspace),
+                                          workspace.numel(), _stream(x.device)))
+    return out
+
+
+def moe_nvfp4_layer_workspace_size(T, H, I, E, K, Is) -> int:
+    return int(_lib().moe_nvfp4_layer_workspace_size(T, H, I, E, K, Is))
+
+
+def moe_nvfp4_layer(x, router_logits, K: int, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
+                    shared_gu, shared_dn, out=None, ids_out=None, w_out=None, workspace=None,
+                    path: int = PATH_AUTO) -> torch.Tensor:
+    """The whole MoE layer in one call: router on the logits, the routed NVFP4 experts,
+    and the BF16 shared expert added before the single rounding to bf16."""
+    _need(x, torch.bfloat16, "x")
+    _need(router_logits, torch.float32, "router_logits")
+    for t, n in ((w_gu, "w_gu"), (s_gu, "s_gu"), (w_dn, "w_dn"), (s_dn, "s_dn")):
+        _need(t, torch.uint8, n)
+    _need(g_gu, torch.float32, "g_gu")
+    _need(g_dn, torch.float32, "g_dn")
+    _need(shared_gu, torch.bfloat16, "shared_gu")
+    _need(shared_dn, torch.bfloat16, "shared_dn")
+    T, H = x.shape
+    E, twoI, _ = w_gu.shape
+    I, Is = twoI // 2, shared_gu.shape[0] // 2
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((moe_nvfp4_layer_workspace_size(T, H, I, E, K, Is),),
+                                dtype=torch.uint8, device=x.device)
+        workspace[:WORKSPACE_ZERO_BYTES].zero_()
+    _check(_lib().moe_nvfp4_layer(
+        _ptr(x), _ptr(router_logits), T, H, I, E, K, _ptr(w_gu), _ptr(s_gu), _ptr(g_gu),
+        _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(shared_gu), _ptr(shared_dn), Is, _ptr(out),
+        _ptr(ids_out), _ptr(w_out), _ptr(workspace), workspace.numel(), int(path),
+        _stream(x.device)))
     return out
 
 

@@ -54,6 +54,8 @@ WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int
   L.y = take(4 * TK * (size_t)H);
   L.xs = take(2 * (TK + kGatherPadRows) * (size_t)H);
   L.xscale = take(4 * TK);
+  L.rids = take(4 * TK);   // router decisions when the call starts from logits
+  L.rw = take(4 * TK);
   L.total = o;
   return L;
 }
@@ -109,18 +111,33 @@ static int64_t local_experts(int64_t E, int64_t size, int64_t rank) {
   return (E - rank + size - 1) / size;
 }
 
+// Where the routing of a forward call comes from: the caller's ids and weights, or the
+// router run on the caller's logits (its decisions written to ids_out / w_out, or to the
+// workspace where those are null).
+struct Routing {
+  const int32_t *ids;
+  const float *w;
+  const float *logits;
+  int32_t *ids_out;
+  float *w_out;
+};
+
 // One forward call.  E is the layer's expert count; `ep_size` > 1 runs the experts of rank
 // `ep_rank` only (the weight arrays then hold those experts) and writes the fp32 partial
 // out_f32 instead of out.
-static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w,
-                        int64_t T, int64_t H, int64_t I, int64_t E, int64_t K, int64_t ep_size,
-                        int64_t ep_rank, const uint8_t *w_gu, const uint8_t *s_gu,
-                        const float *g_gu, const uint8_t *w_dn, const uint8_t *s_dn,
-                        const float *g_dn, __nv_bfloat16 *out, float *out_f32, void *workspace,
-                        size_t ws_bytes, int path, cudaEvent_t const *ev, cudaStream_t stream) {
-  if (!x || !topk_ids || !topk_w || !w_gu || !s_gu || !g_gu || !w_dn || !s_dn || !g_dn ||
-      (!out && !out_f32))
+static int forward_impl(const __nv_bfloat16 *x, const Routing &rt, int64_t T, int64_t H,
+                        int64_t I, int64_t E, int64_t K, int64_t ep_size, int64_t ep_rank,
+                        const uint8_t *w_gu, const uint8_t *s_gu, const float *g_gu,
+                        const uint8_t *w_dn, const uint8_t *s_dn, const float *g_dn,
+                        __nv_bfloat16 *out, float *out_f32, void *workspace, size_t ws_bytes,
+                        int path, cudaEvent_t const *ev, cudaStream_t stream) {
+  if (!x || (!rt.logits && (!rt.ids || !rt.w)) || !w_gu || !s_gu || !g_gu || !w_dn || !s_dn ||
+      !g_dn || (!out && !out_f32))
     return NVFP4_EINVAL;
+  if (rt.logits && (K > E || ((reinterpret_cast<uintptr_t>(rt.logits) |
+                               reinterpret_cast<uintptr_t>(rt.ids_out) |
+                               reinterpret_cast<uintptr_t>(rt.w_out)) & 3)))
+    return K > E ? NVFP4_ESHAPE : NVFP4_EINVAL;
   if (T <= 0 || H <= 0 || I <= 0 || E <= 0 || K <= 0) return NVFP4_EINVAL;
   if (ep_size < 1 || ep_rank < 0 || ep_rank >= ep_size || ep_size > E) return NVFP4_EINVAL;
   if (path != NVFP4_PATH_AUTO && path != NVFP4_PATH_GEMV && path != NVFP4_PATH_GEMM)
@@ -137,8 +154,16 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   char *ws = static_cast<char *>(workspace);
   MoeArgs a = {};
   a.x = x;
-  a.ids = topk_ids;
-  a.w = topk_w;
+  a.ids = rt.ids;
+  a.w = rt.w;
+  int32_t *r_ids = nullptr;   // router output, when the call starts from logits
+  float *r_w = nullptr;
+  if (rt.logits) {
+    r_ids = rt.ids_out ? rt.ids_out : reinterpret_cast<int32_t *>(ws + L.rids);
+    r_w = rt.w_out ? rt.w_out : reinterpret_cast<float *>(ws + L.rw);
+    a.ids = r_ids;
+    a.w = r_w;
+  }
   a.w_gu = w_gu;
   a.s_gu = s_gu;
   a.g_gu = g_gu;
@@ -172,9 +197,11 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
                                                                : NVFP4_PATH_GEMM;
   if (path == NVFP4_PATH_GEMV && !gemv_supported(T, H, I, K)) return NVFP4_ESHAPE;
 
+  if (int s = record(ev, 0, stream)) return s;
+  if (rt.logits)
+    if (int s = launch_router(rt.logits, T, E, K, r_ids, r_w, stream)) return s;
   if (path == NVFP4_PATH_GEMV) {
     // routing is recomputed inside each projection kernel, so there is no route launch
-    if (int s = record(ev, 0, stream)) return s;
     if (int s = record(ev, 1, stream)) return s;
     if (int s = launch_gemv_gateup(a, stream)) return s;
     if (int s = record(ev, 2, stream)) return s;
@@ -186,7 +213,7 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   }
 
   RouteArgs r = {};
-  r.ids = topk_ids;
+  r.ids = a.ids;
   r.n_pairs = T * K;
   r.E = (int)E_loc;
   r.map = a.map;
@@ -199,7 +226,6 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   r.n_active = a.n_active;
   r.tile_prefix = a.tile_prefix;
   r.tile_n = gemm_tile_n();
-  if (int s = record(ev, 0, stream)) return s;
   if (int s = launch_route(r, stream, true)) return s;
   if (int s = record(ev, 1, stream)) return s;
   if (int s = launch_gemm_gateup(a, stream)) return s;
@@ -210,6 +236,20 @@ static int forward_impl(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   return record(ev, 4, stream);
 }
 
+namespace nvfp4 {
+int forward_logits_partial(const __nv_bfloat16 *x, const float *logits, int64_t T, int64_t H,
+                           int64_t I, int64_t E, int64_t K, const uint8_t *w_gu,
+                           const uint8_t *s_gu, const float *g_gu, const uint8_t *w_dn,
+                           const uint8_t *s_dn, const float *g_dn, float *out_f32,
+                           int32_t *ids_out, float *w_out, void *workspace, size_t ws_bytes,
+                           int path, cudaStream_t stream) {
+  if (!logits || !out_f32) return NVFP4_EINVAL;
+  const Routing rt = {nullptr, nullptr, logits, ids_out, w_out};
+  return forward_impl(x, rt, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, nullptr,
+                      out_f32, workspace, ws_bytes, path, nullptr, stream);
+}
+}  // namespace nvfp4
+
 extern "C" int moe_nvfp4_forward_path(const __nv_bfloat16 *x, const int32_t *topk_ids,
                                       const float *topk_w, int64_t T, int64_t H, int64_t I,
                                       int64_t E, int64_t K, const uint8_t *w_gu,
@@ -217,8 +257,9 @@ extern "C" int moe_nvfp4_forward_path(const __nv_bfloat16 *x, const int32_t *top
                                       const uint8_t *w_dn, const uint8_t *s_dn,
                                       const float *g_dn, __nv_bfloat16 *out, void *workspace,
                                       size_t ws_bytes, int path, cudaStream_t stream) {
-  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn,
-                      g_dn, out, nullptr, workspace, ws_bytes, path, nullptr, stream);
+  const Routing rt = {topk_ids, topk_w, nullptr, nullptr, nullptr};
+  return forward_impl(x, rt, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, out,
+                      nullptr, workspace, ws_bytes, path, nullptr, stream);
 }
 
 extern "C" int moe_nvfp4_forward_profiled(const __nv_bfloat16 *x, const int32_t *topk_ids,
@@ -232,8 +273,9 @@ extern "C" int moe_nvfp4_forward_profiled(const __nv_bfloat16 *x, const int32_t 
   if (!stage_events) return NVFP4_EINVAL;
   for (int i = 0; i < 5; ++i)
     if (!stage_events[i]) return NVFP4_EINVAL;
-  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn,
-                      g_dn, out, nullptr, workspace, ws_bytes, path,
+  const Routing rt = {topk_ids, topk_w, nullptr, nullptr, nullptr};
+  return forward_impl(x, rt, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, out,
+                      nullptr, workspace, ws_bytes, path,
                       reinterpret_cast<cudaEvent_t const *>(stage_events), stream);
 }
 
@@ -259,9 +301,23 @@ extern "C" int moe_nvfp4_forward_ep(const __nv_bfloat16 *x, const int32_t *topk_
                                     float *out_partial, void *workspace, size_t ws_bytes,
                                     int path, cudaStream_t stream) {
   if (!out_partial) return NVFP4_EINVAL;
-  return forward_impl(x, topk_ids, topk_w, T, H, I, E, K, ep_size, ep_rank, w_gu, s_gu, g_gu,
-                      w_dn, s_dn, g_dn, nullptr, out_partial, workspace, ws_bytes, path,
-                      nullptr, stream);
+  const Routing rt = {topk_ids, topk_w, nullptr, nullptr, nullptr};
+  return forward_impl(x, rt, T, H, I, E, K, ep_size, ep_rank, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn,
+                      nullptr, out_partial, workspace, ws_bytes, path, nullptr, stream);
+}
+
+extern "C" int moe_nvfp4_forward_logits(const __nv_bfloat16 *x, const float *router_logits,
+                                        int64_t T, int64_t H, int64_t I, int64_t E, int64_t K,
+                                        const uint8_t *w_gu, const uint8_t *s_gu,
+                                        const float *g_gu, const uint8_t *w_dn,
+                                        const uint8_t *s_dn, const float *g_dn,
+                                        __nv_bfloat16 *out, int32_t *topk_ids_out,
+                                        float *topk_w_out, void *workspace, size_t ws_bytes,
+                                        int path, cudaStream_t stream) {
+  if (!router_logits) return NVFP4_EINVAL;
+  const Routing rt = {nullptr, nullptr, router_logits, topk_ids_out, topk_w_out};
+  return forward_impl(x, rt, T, H, I, E, K, 1, 0, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, out,
+                      nullptr, workspace, ws_bytes, path, nullptr, stream);
 }
 
 extern "C" int moe_nvfp4_read_error_flag(const void *workspace, int32_t *host_flag,

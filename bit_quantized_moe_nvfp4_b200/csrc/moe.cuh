@@ -41,7 +41,8 @@ struct MoeArgs {
 
 // Workspace carve-up (byte offsets, each 256-aligned).
 struct WorkspaceLayout {
-  size_t flag, work, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, xscale, total;
+  size_t flag, work, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, xscale,
+      rids, rw, total;
 };
 WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
 constexpr int kGatherPadRows = 256;
@@ -51,6 +52,17 @@ bool gemv_supported(int64_t T, int64_t H, int64_t I, int64_t K);
 int launch_gemv_gateup(const MoeArgs &a, cudaStream_t s);
 int launch_gemv_down(const MoeArgs &a, cudaStream_t s);
 bool gemv_fused_combine(int64_t T);   // the GEMV down kernel also combines (no combine launch)
+// The routed layer from router logits with its fp32 sum (before the bf16 rounding) written
+// to out_f32 (api.cu); the shared expert's down step adds to it and rounds.
+int forward_logits_partial(const __nv_bfloat16 *x, const float *logits, int64_t T, int64_t H,
+                           int64_t I, int64_t E, int64_t K, const uint8_t *w_gu,
+                           const uint8_t *s_gu, const float *g_gu, const uint8_t *w_dn,
+                           const uint8_t *s_dn, const float *g_dn, float *out_f32,
+                           int32_t *ids_out, float *w_out, void *workspace, size_t ws_bytes,
+                           int path, cudaStream_t stream);
+// router (router.cu): top-K of each token's E logits, renormalised softmax weights
+int launch_router(const float *logits, int64_t T, int64_t E, int64_t K, int32_t *ids, float *w,
+                  cudaStream_t s);
 // combine of the GEMM path (combine.cu)
 int launch_combine(const MoeArgs &a, cudaStream_t s);
 int launch_combine_pairs(const MoeArgs &a, cudaStream_t s);   // y indexed by pair (GEMV path)

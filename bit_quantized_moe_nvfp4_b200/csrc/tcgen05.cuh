@@ -5,6 +5,8 @@
 // stored at chunk position c ^ (r % 8).  Accumulators live in tensor memory (TMEM): lane =
 // row of D, column = column of D, 32-bit cells.
 #pragma once
+#include <cuda.h>
+
 #include "pipeline.cuh"
 
 namespace nvfp4 {
@@ -138,6 +140,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 }
 
 // ---------------------------------------------------------------- TMA (tiled, 2-D)
+// Host: a 2-D tiled tensor map over a row-major [rows, cols] array of elem_bytes-sized
+// elements, boxes of box_rows x box_cols (gemm.cu).  NVFP4_OK, or NVFP4_ECUDA if the driver
+// refuses it.
+int make_map(CUtensorMap *m, CUtensorMapDataType type, int elem_bytes, const void *base,
+             uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+             CUtensorMapSwizzle swz);
+
 // Load the box at coordinates (x, y) of the tensor map into shared memory, completing the
 // transferred bytes on `bar`.  x * element size must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y,

@@ -198,6 +198,80 @@ NVFP4_API int moe_nvfp4_forward_profiled(const __nv_bfloat16 *x, const int32_t *
                                          void *workspace, size_t ws_bytes, int path,
                                          void *const *stage_events, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- router */
+
+/* The router's decision for each token (page "GLM-5-NVFP4-MTP", "Model Description":
+ * 256 experts, 8 active per token; the router stays BF16 / fp32 per "What's quantized").
+ * The pages do not state its function; the one computed is: p = softmax(logits[t, :]),
+ * the K largest p in descending order with the lower expert index first among equal
+ * values, and their weights p_k / (sum of the K selected p).  The selection compares the
+ * fp32 logits themselves (softmax preserves their order), so it is exact; the weights are
+ * fp32, exp(l_k - l_max) / sum of exp(l_j - l_max) over the selected j.
+ *   logits    [T, E] fp32, finite (NaN or infinite logits give unspecified results)
+ *   topk_ids  [T, K] int32 out: slot k = the k-th largest logit's expert
+ *   topk_w    [T, K] fp32 out: positive, summing to 1 over a token's K slots
+ * Limits: 1 <= K <= min(16, E), E <= 1024, T*K < 2^31.  Pointers 4-byte aligned.
+ * Errors: EINVAL, ESHAPE, ECUDA. */
+NVFP4_API int moe_nvfp4_router(const float *logits, int64_t T, int64_t E, int64_t K,
+                               int32_t *topk_ids, float *topk_w, cudaStream_t stream);
+
+/* moe_nvfp4_forward_path from router logits: the router above, then the layer on its
+ * decisions (one stream-ordered chain, no host round trip).  topk_ids_out / topk_w_out
+ * ([T, K], may be NULL) receive the decisions; when NULL they stay in the workspace.
+ * Arguments, layouts, limits and errors otherwise as moe_nvfp4_forward_path (plus ESHAPE
+ * for K > E). */
+NVFP4_API int moe_nvfp4_forward_logits(const __nv_bfloat16 *x, const float *router_logits,
+                                       int64_t T, int64_t H, int64_t I, int64_t E, int64_t K,
+                                       const uint8_t *w_gu, const uint8_t *s_gu,
+                                       const float *g_gu, const uint8_t *w_dn,
+                                       const uint8_t *s_dn, const float *g_dn,
+                                       __nv_bfloat16 *out, int32_t *topk_ids_out,
+                                       float *topk_w_out, void *workspace, size_t ws_bytes,
+                                       int path, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- shared expert, layer */
+
+/* The shared expert: a dense SwiGLU MLP in BF16 that every token passes through beside the
+ * routed experts (page "GLM-5-NVFP4-MTP", "What's quantized": only the routed experts are
+ * NVFP4; the rest of the model, shared experts included, stays BF16).  For every token t:
+ *   h[t, j]   = bf16( silu(w_gu[j] . x_t) * (w_gu[Is + j] . x_t) )      j < Is
+ *   out[t, n] = bf16( routed[t, n] + w_dn[n] . h[t] )                     n < H
+ * with exact bf16 products and fp32 sums (the order of the fp32 sums is the kernel's).
+ *   x       [T, H] bf16              w_gu [2 Is, H] bf16 (gate rows, then up rows)
+ *   w_dn    [H, Is] bf16             routed [T, H] fp32, or NULL for 0 (e.g. the partial
+ *                                    of moe_nvfp4_forward_ep, or a reduced sum of them)
+ *   out     [T, H] bf16
+ * Limits: H % 64 == 0, Is % 64 == 0, H and Is <= 65536; with T <= 8 the tokens' rows must
+ * fit one CTA's shared memory (T * max(H, Is) * 2 bytes <= 227 KB, else ESHAPE).
+ * Alignment: x, w_gu, w_dn, out and workspace 16 bytes; routed 4 bytes.
+ * Workspace: moe_nvfp4_shared_workspace_size(T, Is) bytes (holds h), no initialisation.
+ * Errors: EINVAL, ESHAPE, EWORKSPACE, ECUDA. */
+NVFP4_API size_t moe_nvfp4_shared_workspace_size(int64_t T, int64_t Is);
+NVFP4_API int moe_nvfp4_shared_expert(const __nv_bfloat16 *x, int64_t T, int64_t H, int64_t Is,
+                                      const __nv_bfloat16 *w_gu, const __nv_bfloat16 *w_dn,
+                                      const float *routed, __nv_bfloat16 *out, void *workspace,
+                                      size_t ws_bytes, cudaStream_t stream);
+
+/* The whole MoE layer in one stream-ordered call: the router on router_logits
+ * (moe_nvfp4_router), the routed NVFP4 experts summed in fp32 (moe_nvfp4_forward_logits
+ * before its rounding), and the shared expert added to that sum before the single rounding
+ * to bf16:  out[t] = bf16( sum_k w[t,k] y_k(t) + shared(x_t) ).
+ * Arguments as moe_nvfp4_forward_logits plus shared_gu [2 Is, H] / shared_dn [H, Is] bf16
+ * and Is; limits of both.  Workspace: moe_nvfp4_layer_workspace_size bytes whose first
+ * NVFP4_WORKSPACE_ZERO_BYTES are zero before its first use (the error flag, read with
+ * moe_nvfp4_read_error_flag, is its first word).  Errors: EINVAL, ESHAPE, EWORKSPACE,
+ * ECUDA. */
+NVFP4_API size_t moe_nvfp4_layer_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E,
+                                                int64_t K, int64_t Is);
+NVFP4_API int moe_nvfp4_layer(const __nv_bfloat16 *x, const float *router_logits, int64_t T,
+                              int64_t H, int64_t I, int64_t E, int64_t K, const uint8_t *w_gu,
+                              const uint8_t *s_gu, const float *g_gu, const uint8_t *w_dn,
+                              const uint8_t *s_dn, const float *g_dn,
+                              const __nv_bfloat16 *shared_gu, const __nv_bfloat16 *shared_dn,
+                              int64_t Is, __nv_bfloat16 *out, int32_t *topk_ids_out,
+                              float *topk_w_out, void *workspace, size_t ws_bytes, int path,
+                              cudaStream_t stream);
+
 /* Copy the workspace error flag to *host_flag (host pointer) and wait for it:
  * 0 = no error, bit 0 = an id outside [0, E) was met, bit 1 = a device-side wait gave up.
  * The flag is cleared by the next moe_nvfp4_forward on that workspace.  Synchronises

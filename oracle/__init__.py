@@ -76,6 +76,12 @@ def _load():
             L.oracle_nvfp4_dequantize.argtypes = [P, P, P, I64, I64, I64, P]
             L.oracle_route.restype = I64
             L.oracle_route.argtypes = [P, I64, I64, I64, P, P, P, P]
+            L.oracle_shared_expert.restype = None
+            L.oracle_shared_expert.argtypes = [P, I64, I64, P, P, P, I64, P]
+            L.oracle_bf16_round_array.restype = None
+            L.oracle_bf16_round_array.argtypes = [P, I64, P]
+            L.oracle_router.restype = None
+            L.oracle_router.argtypes = [P, I64, I64, I64, P, P]
             L.oracle_moe_forward.restype = I64
             L.oracle_moe_forward.argtypes = [P, P, P, I64, I64, I64, I64, I64,
                                              P, P, P, P, P, P, P, I64, P, P]
@@ -217,6 +223,18 @@ def route(ids, E: int):
     return counts, offsets, perm[: offsets[E]], inv, int(bad)
 
 
+def router(logits, K: int):
+    """Router decisions from fp32 logits [T, E]: (ids int32 [T, K], w fp64 [T, K])."""
+    a = _np(logits, np.float32)
+    T, E = a.shape
+    if not 1 <= K <= E:
+        raise ValueError(f"K={K} outside 1..{E}")
+    ids = np.zeros((T, K), np.int32)
+    w = np.zeros((T, K), np.float64)
+    _load().oracle_router(_p(a), T, E, K, _p(ids), _p(w))
+    return ids, w
+
+
 # ----------------------------------------------------------------------------- MoE
 def moe_forward(x, ids, w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, tokens=None):
     """Routed-expert MoE forward for the listed tokens (all when tokens is None).
@@ -243,6 +261,28 @@ def moe_forward(x, ids, w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, tokens=None):
                                      _p(pg), _p(sg), _p(gg), _p(pd), _p(sd), _p(gd),
                                      _p(tok), tok.size, _p(out), _p(out64))
     return out, out64, int(bad)
+
+
+def shared_expert(x, w_gu, w_dn, tokens=None):
+    """Shared-expert output y fp64 [n_tok, H] for the listed tokens (all when None).
+    x bf16 [T, H]; w_gu bf16 [2Is, H]; w_dn bf16 [H, Is] (torch bf16 tensors or uint16)."""
+    xs, gu, dn = _u16(x), _u16(w_gu), _u16(w_dn)
+    T, H = xs.shape
+    Is = gu.shape[0] // 2
+    if gu.shape != (2 * Is, H) or dn.shape != (H, Is):
+        raise ValueError("w_gu [2Is, H] and w_dn [H, Is]")
+    tok = np.arange(T, dtype=np.int64) if tokens is None else np.asarray(tokens, np.int64)
+    y = np.zeros((tok.size, H), np.float64)
+    _load().oracle_shared_expert(_p(xs), H, Is, _p(gu), _p(dn), _p(tok), tok.size, _p(y))
+    return y
+
+
+def bf16_round_array(v) -> np.ndarray:
+    """bf16 bits (uint16) of the fp64 values v, each rounded once to nearest even."""
+    a = np.ascontiguousarray(v, np.float64)
+    out = np.zeros(a.shape, np.uint16)
+    _load().oracle_bf16_round_array(_p(a), a.size, _p(out))
+    return out
 
 
 def bf16_bits_to_f32(u16: np.ndarray) -> np.ndarray:

@@ -333,6 +333,54 @@ int64_t oracle_route(const int32_t *ids, int64_t T, int64_t K, int64_t E,
 }
 
 /* ------------------------------------------------------------------------------------- */
+/* Router                                                                                */
+/* ------------------------------------------------------------------------------------- */
+
+/* The router's decision per token.  Page "GLM-5-NVFP4-MTP", "Model Description": each
+ * token is served by 8 of the 256 experts; "What's quantized" keeps the router in BF16/fp32.
+ * The pages do not give the router's function.  Reading taken: p = softmax(logits[t, :]),
+ * the K experts of largest p, in descending order of p with the lower index first among
+ * equal p, and weights w_k = p_k / (sum of the K selected p).
+ * Which p is larger is decided on the fp32 logits, which is the exact order of the
+ * real-valued softmax (it is strictly increasing in the logit).  Comparing the fp64-rounded
+ * p instead would create false ties where exp underflows or where l - max rounds to the
+ * same double.  The weights follow the definition in fp64: softmax over all E, then
+ * renormalisation over the selected K.
+ *   logits [T, E] fp32  ->  ids [T, K] int32, w [T, K] fp64                              */
+void oracle_router(const float *logits, int64_t T, int64_t E, int64_t K, int32_t *ids,
+                   double *w)
+{
+    double *p = (double *)malloc((size_t)E * sizeof(double));
+    unsigned char *taken = (unsigned char *)malloc((size_t)E);
+    for (int64_t t = 0; t < T; ++t) {
+        const float *l = logits + t * E;
+        double m = -INFINITY;
+        for (int64_t e = 0; e < E; ++e)
+            if ((double)l[e] > m) m = (double)l[e];
+        double z = 0.0;
+        for (int64_t e = 0; e < E; ++e) {
+            p[e] = exp((double)l[e] - m);
+            z += p[e];
+        }
+        for (int64_t e = 0; e < E; ++e) p[e] = p[e] / z;
+        memset(taken, 0, (size_t)E);
+        double s = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; ++e)   /* strict >: the lower index wins a tie */
+                if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+            taken[best] = 1;
+            ids[t * K + k] = (int32_t)best;
+            w[t * K + k] = p[best];
+            s += p[best];
+        }
+        for (int64_t k = 0; k < K; ++k) w[t * K + k] = w[t * K + k] / s;
+    }
+    free(p);
+    free(taken);
+}
+
+/* ------------------------------------------------------------------------------------- */
 /* MoE forward                                                                           */
 /* ------------------------------------------------------------------------------------- */
 
@@ -418,6 +466,51 @@ int64_t oracle_moe_forward(const uint16_t *x, const int32_t *ids, const float *w
     free(hb);
     free(acc);
     return bad;
+}
+
+/* The shared expert: a dense SwiGLU MLP in BF16 that every token passes through, next to
+ * the routed experts.  Page "GLM-5-NVFP4-MTP", "What's quantized": only the routed
+ * experts' projections are NVFP4 and everything else stays BF16.  A page on the same model
+ * family lists the shared experts among its BF16 tensors.  For the tokens tok[0..n_tok):
+ *   a   = Wgu x_t                        (2 Is values; rows 0..Is-1 gate, Is..2Is-1 up)
+ *   h_j = bf16( silu(a_j) * a_{Is+j} )   (rounded to bf16, as for the routed experts)
+ *   y   = Wdn h                          (H values)
+ * in fp64 with the bf16 weights exactly.  The layer output is bf16(routed sum + y).
+ * [Reading: the shared expert's output is added with weight 1; the pages give no scale.]
+ * Shapes: x [T,H] bf16, Wgu [2Is,H] bf16, Wdn [H,Is] bf16; y [n_tok,H] fp64. */
+void oracle_shared_expert(const uint16_t *x, int64_t H, int64_t Is, const uint16_t *wgu,
+                          const uint16_t *wdn, const int64_t *tok, int64_t n_tok, double *y)
+{
+    double *xt = (double *)malloc(sizeof(double) * H);
+    double *a = (double *)malloc(sizeof(double) * 2 * Is);
+    double *hb = (double *)malloc(sizeof(double) * Is);
+    for (int64_t i = 0; i < n_tok; ++i) {
+        int64_t t = tok[i];
+        for (int64_t c = 0; c < H; ++c) xt[c] = oracle_bf16_to_f32(x[t * H + c]);
+        #pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < 2 * Is; ++j) {
+            double s = 0.0;
+            for (int64_t c = 0; c < H; ++c) s += oracle_bf16_to_f32(wgu[j * H + c]) * xt[c];
+            a[j] = s;
+        }
+        for (int64_t j = 0; j < Is; ++j)
+            hb[j] = oracle_bf16_to_f32(oracle_bf16_round(silu(a[j]) * a[Is + j]));
+        #pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < H; ++n) {
+            double s = 0.0;
+            for (int64_t c = 0; c < Is; ++c) s += oracle_bf16_to_f32(wdn[n * Is + c]) * hb[c];
+            y[i * H + n] = s;
+        }
+    }
+    free(xt);
+    free(a);
+    free(hb);
+}
+
+/* out[i] = bf16(v[i]) for n values (the layer's final rounding of an fp64 sum). */
+void oracle_bf16_round_array(const double *v, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_round(v[i]);
 }
 
 /* Number of OpenMP threads the oracle's parallel loops use (1 without OpenMP). */

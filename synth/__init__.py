@@ -1,9 +1,12 @@
 """Seeded synthetic inputs for the NVFP4 MoE layer.
 
-This module only makes data: bf16 weights and activations drawn from normal laws, and
-routing decisions (softmax over random router logits, top-k, renormalised).  It holds
-none of the method's arithmetic (no quantisation, no expert math), so both the CUDA
-path and the CPU oracle may take their inputs from it.
+This module only makes data: bf16 weights and activations drawn from normal laws, router
+logits, and routing decisions for the routed-expert tests.  It holds none of the method's
+arithmetic (no quantisation, no expert math), so both the CUDA path and the CPU oracle may
+take their inputs from it.  routing() turns random logits into (ids, weights) with numpy
+and torch in fp64 so that the layer's inputs look like a router's output; the library's
+own router is tested only on router_logits() against the oracle's router, never against
+routing().
 
 Workloads follow the routed-expert MoE of page "GLM-5-NVFP4-MTP", "Model Description"
 (256 experts, 8 active per token) at hidden size 6144 and expert intermediate size 2048:
@@ -71,6 +74,17 @@ def expert_weights_bf16(E: int, H: int, I: int, seed: int, device="cpu", std: fl
 
 def activations_bf16(T: int, H: int, seed: int, device="cpu") -> torch.Tensor:
     return normal_bf16((T, H), seed, "x", device=device)
+
+
+def router_logits(T: int, E: int, seed: int, zipf_bias: float = 0.0) -> torch.Tensor:
+    """Router logits fp32 [T, E] on the CPU: N(0,1) + zipf_bias * ln(1/(e+1)), rounded to
+    fp32 (the same draw as routing() with the same seed)."""
+    g = _gen("cpu", seed, "router")
+    logits = torch.randn((T, E), generator=g, dtype=torch.float64)
+    if zipf_bias:
+        e = torch.arange(E, dtype=torch.float64)
+        logits = logits + zipf_bias * torch.log(1.0 / (e + 1.0))
+    return logits.float()
 
 
 def routing(T: int, E: int, K: int, seed: int, zipf_bias: float = 0.0):

@@ -191,6 +191,35 @@ def test_expert_parallel_argument_checks_run_before_cuda(lib):
     assert red(ptrs, 2, 0, 8, fake, None) == 0          # no rows: nothing to enqueue
 
 
+def test_router_argument_checks_run_before_cuda(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    r = lib.moe_nvfp4_router
+    r.restype = ctypes.c_int
+    r.argtypes = [P, I64, I64, I64, P, P, P]
+    fake = ctypes.c_void_p(1 << 20)
+    assert r(None, 4, 256, 8, fake, fake, None) == -1
+    assert r(fake, 0, 256, 8, fake, fake, None) == -1
+    assert r(fake, 4, 256, 0, fake, fake, None) == -1
+    assert r(fake, 4, 256, 17, fake, fake, None) == -2
+    assert r(fake, 4, 4, 5, fake, fake, None) == -2          # K > E
+    assert r(fake, 4, 2048, 8, fake, fake, None) == -2
+    assert r(ctypes.c_void_p((1 << 20) + 2), 4, 256, 8, fake, fake, None) == -1
+    f = lib.moe_nvfp4_forward_logits
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, I64, I64, I64, I64, I64, P, P, P, P, P, P, P, P, P, P,
+                  ctypes.c_size_t, ctypes.c_int, P]
+
+    def call(logits=fake, ws_bytes=1 << 40, **over):
+        d = dict(dict(T=1, H=6144, I=2048, E=256, K=8), **over)
+        return f(fake, logits, d["T"], d["H"], d["I"], d["E"], d["K"], fake, fake, fake, fake,
+                 fake, fake, fake, None, None, fake, ws_bytes, 0, None)
+
+    assert call(logits=None) == -1
+    assert call(E=4, K=8) == -2
+    assert call(H=6100) == -2
+    assert call(ws_bytes=16) == -3
+
+
 def test_selftest_argument_checks_run_before_cuda(lib):
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f = lib.nvfp4_selftest_wait_timeout

@@ -365,3 +365,122 @@ def test_calibrated_range_invariants(factor):
         # below one E2M1 step of the block
         scl = np.repeat(np.vectorize(oracle.e4m3_value)(s), 16, axis=2) * g[:, None, None]
         assert np.all(np.abs(deq - xf) <= scl * 2.0 + 1e-30)
+
+
+# ----------------------------------------------------------------------------- router
+# Page "GLM-5-NVFP4-MTP", "Model Description" (8 of 256 experts per token); reading: softmax
+# -> K largest (lower index first on ties) -> renormalised over the K.
+
+def test_router_equal_logits_pick_the_lowest_indices():
+    ids, w = oracle.router(np.zeros((2, 10), np.float32) + np.float32(0.7), 4)
+    assert ids.tolist() == [[0, 1, 2, 3]] * 2
+    np.testing.assert_allclose(w, 0.25, rtol=0, atol=1e-15)
+
+
+def test_router_two_value_closed_form():
+    # softmax([0, ln 3]) = [1/4, 3/4]; with K = E nothing is dropped
+    ids, w = oracle.router(np.array([[0.0, np.log(3.0)]], np.float32), 2)
+    assert ids.tolist() == [[1, 0]]
+    l1 = float(np.float32(np.log(3.0)))
+    want = np.array([np.exp(l1), 1.0]) / (1.0 + np.exp(l1))
+    np.testing.assert_allclose(w[0], want, rtol=1e-15)
+    np.testing.assert_allclose(w[0], [0.75, 0.25], rtol=1e-7)
+
+
+def test_router_hand_example_with_a_tie():
+    # logits [1, 3, 2, 3]: experts 1 and 3 tie at the top (1 first), then 2;
+    # weights e^3 : e^3 : e^2 renormalised = e/(2e+1), e/(2e+1), 1/(2e+1)
+    ids, w = oracle.router(np.array([[1.0, 3.0, 2.0, 3.0]], np.float32), 3)
+    assert ids.tolist() == [[1, 3, 2]]
+    e = np.e
+    np.testing.assert_allclose(w[0], [e / (2 * e + 1), e / (2 * e + 1), 1 / (2 * e + 1)],
+                               rtol=1e-14)
+
+
+def test_router_top1_has_weight_one():
+    logits = synth.router_logits(50, 37, seed=4)
+    ids, w = oracle.router(logits, 1)
+    assert np.array_equal(ids[:, 0], np.argmax(logits.numpy(), axis=1))
+    assert np.all(w == 1.0)
+
+
+def test_router_underflowed_probabilities_keep_the_logit_order():
+    # exp(-1000) and below underflow to 0 in fp64: the order still follows the logits
+    ids, w = oracle.router(np.array([[0.0, -1000.0, -2000.0, -1500.0]], np.float32), 3)
+    assert ids.tolist() == [[0, 1, 3]]
+    assert w.tolist() == [[1.0, 0.0, 0.0]]
+
+
+def test_router_shift_invariant():
+    logits = synth.router_logits(20, 64, seed=9, zipf_bias=1.5)
+    ids0, w0 = oracle.router(logits, 8)
+    ids1, w1 = oracle.router(logits + 8.0, 8)   # exact: |logits| < 8, shifts of 8 keep order
+    assert np.array_equal(ids0, ids1)
+    np.testing.assert_allclose(w0, w1, rtol=1e-5)
+
+
+def test_router_matches_stable_argsort_and_topk_softmax():
+    """Brute force by another route: numpy's stable argsort of -logits for the choice, and
+    the softmax of the K chosen logits alone for the weights (the full denominator cancels
+    in the renormalisation)."""
+    for T, E, K, bias in ((64, 8, 2, 0.0), (33, 256, 8, 1.5), (5, 1024, 16, 0.0)):
+        logits = synth.router_logits(T, E, seed=E + K, zipf_bias=bias).numpy()
+        ids, w = oracle.router(logits, K)
+        want = np.argsort(-logits, axis=1, kind="stable")[:, :K]
+        assert np.array_equal(ids, want)
+        top = np.take_along_axis(logits.astype(np.float64), want, axis=1)
+        ex = np.exp(top - top[:, :1])
+        np.testing.assert_allclose(w, ex / ex.sum(axis=1, keepdims=True), rtol=1e-12)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-14)
+
+
+# ----------------------------------------------------------------------------- shared expert
+# Page "GLM-5-NVFP4-MTP", "What's quantized": every weight but the routed experts' stays
+# BF16; the shared expert is a dense SwiGLU MLP added to the routed sum.
+
+def test_shared_expert_identity_weights():
+    """Gate = identity, up = 2 x identity, down = identity: y_n = bf16(silu(x_n) * 2 x_n).
+    Exchanging gate and up would give silu(2 x) * x instead."""
+    H = Is = 64
+    eye = torch.eye(H, dtype=torch.float32)
+    w_gu = torch.cat([eye, 2 * eye]).to(torch.bfloat16)
+    w_dn = eye.to(torch.bfloat16)
+    x = torch.linspace(-4, 4, H).view(1, H).to(torch.bfloat16)
+    y = oracle.shared_expert(x, w_gu, w_dn)
+    xv = x.double().numpy()[0]
+    want = oracle.bf16_bits_to_f32(oracle.bf16_round_array(xv / (1 + np.exp(-xv)) * 2 * xv))
+    np.testing.assert_array_equal(y[0], want.astype(np.float64))
+    swapped = 2 * xv / (1 + np.exp(-2 * xv)) * xv
+    assert np.abs(y[0] - swapped).max() > 0.1
+
+
+def test_shared_expert_matches_dense_brute_force():
+    T, H, Is = 5, 128, 64
+    x = synth.activations_bf16(T, H, 3)
+    w_gu = synth.normal_bf16((2 * Is, H), 3, "sgu", std=0.05)
+    w_dn = synth.normal_bf16((H, Is), 3, "sdn", std=0.05)
+    y = oracle.shared_expert(x, w_gu, w_dn)
+    X, G, D = (t.double().numpy() for t in (x, w_gu, w_dn))
+    a = X @ G.T
+    hh = a[:, :Is] / (1 + np.exp(-a[:, :Is])) * a[:, Is:]
+    h = oracle.bf16_bits_to_f32(oracle.bf16_round_array(hh)).astype(np.float64)
+    np.testing.assert_allclose(y, h @ D.T, rtol=1e-12, atol=1e-12)
+    # a subset of tokens gives the same rows
+    np.testing.assert_array_equal(oracle.shared_expert(x, w_gu, w_dn, tokens=[4, 1]), y[[4, 1]])
+
+
+def test_shared_expert_zero_input_and_down_linearity():
+    H, Is = 64, 128
+    w_gu = synth.normal_bf16((2 * Is, H), 5, "sgu", std=0.05)
+    w_dn = synth.normal_bf16((H, Is), 5, "sdn", std=0.05)
+    assert np.all(oracle.shared_expert(torch.zeros(2, H, dtype=torch.bfloat16), w_gu, w_dn) == 0)
+    x = synth.activations_bf16(3, H, 5)
+    y1 = oracle.shared_expert(x, w_gu, w_dn)
+    y2 = oracle.shared_expert(x, w_gu, (w_dn.float() * 2).to(torch.bfloat16))
+    np.testing.assert_array_equal(y2, 2 * y1)
+
+
+def test_bf16_round_array_matches_scalar_rounding():
+    v = np.concatenate([synth.router_logits(4, 64, seed=1).double().numpy().ravel() * 1e3,
+                        [0.0, -0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9, 65504.0]])
+    assert [int(b) for b in oracle.bf16_round_array(v)] == [oracle.bf16_round(x) for x in v]
