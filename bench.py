@@ -2,7 +2,7 @@
 """Benchmark of the NVFP4 routed-expert MoE layer on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload all|prefill|decode1|decode8|decode32|decode64|codec]
+                    [--workload all|prefill|decode1|decode8|decode32|decode64|codec|layer]
 
 A step is one pass of the whole layer (route -> gate/up + SwiGLU -> down -> combine) over
 one batch of the H=6144, I=2048, E=256, top-8 layer whose NVFP4 weights (5.4 GB, N(0,0.02)
@@ -594,12 +594,142 @@ class Bench:
                 **res}
 
 
+SHARED_I = I                  # shared-expert intermediate size (one expert's, 2048)
+SHARED_BYTES = 3 * H * SHARED_I * 2     # bf16 gate, up and down weights: 75.5 MB
+SHARED_COPIES = 3                       # rotated so the 75.5 MB are not left in L2
+
+
+def graph_timed(stream, fn, n_calls, steps, warmup):
+    """Time `steps` calls of fn(i) (i cycles over n_calls prepared inputs) replayed from a
+    CUDA graph of n_calls calls; returns (ms per call, clock summary)."""
+    for i in range(warmup):
+        fn(i % n_calls)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn(0)
+        stream.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(n_calls):
+                fn(i)
+    reps = max(1, steps // n_calls)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device(), stream, graph.replay) as clk:
+        torch.cuda.synchronize()
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * n_calls)
+    del graph
+    return ms, clk.summary()
+
+
+def shared_layer_records(b, warmup):
+    """The BF16 shared expert alone and the whole layer (router + routed NVFP4 experts +
+    shared expert, moe_nvfp4_layer) at one token and at the T = 4096 prefill batch."""
+    nv, device, peaks = b.nv, b.device, b.peaks
+    layer = b.ensure_layer()
+    stream = torch.cuda.Stream(device)
+    shared = [(synth.normal_bf16((2 * SHARED_I, H), c, "shared_gu", std=0.02, device=device),
+               synth.normal_bf16((H, SHARED_I), c, "shared_dn", std=0.02, device=device))
+              for c in range(SHARED_COPIES)]
+    recs = []
+    for T, steps, n_calls in ((1, 2048, 256), (4096, 10, 2)):
+        wl = synth.PREFILL_T4096 if T > 1 else synth.DECODE_T1
+        xs = synth.activations_bf16(n_calls * T, H, 31, device=device).view(n_calls, T, H)
+        logits = synth.router_logits(n_calls * T, E, seed=31, zipf_bias=wl.zipf_bias)
+        logits = logits.view(n_calls, T, E).to(device)
+        routed = torch.randn(T, H, device=device) * 0.05
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        sws = torch.empty((max(16, T * SHARED_I * 2),), dtype=torch.uint8, device=device)
+        lws = torch.zeros((nv.moe_nvfp4_layer_workspace_size(T, H, I, E, K, SHARED_I),),
+                          dtype=torch.uint8, device=device)
+
+        def shared_call(i):
+            gu, dn = shared[i % SHARED_COPIES]
+            nv.moe_nvfp4_shared_expert(xs[i], gu, dn, routed=routed, out=out, workspace=sws)
+
+        def layer_call(i):
+            gu, dn = shared[i % SHARED_COPIES]
+            nv.moe_nvfp4_layer(xs[i], logits[i], K, *layer, gu, dn, out=out, workspace=lws)
+
+        ms_s, clk_s = graph_timed(stream, shared_call, n_calls, steps, warmup)
+        ms_l, clk_l = graph_timed(stream, layer_call, n_calls, steps, warmup)
+        ids = torch.stack([nv.moe_nvfp4_router(logits[i], K)[0] for i in range(n_calls)])
+        uniq = statistics.mean(len(set(ids[i].flatten().tolist())) for i in range(n_calls))
+        if T == 1:
+            ach_s = SHARED_BYTES / (ms_s / 1e3) / 1e9
+            roof_s = {"kernel": "shared_gemv_gateup + shared_gemv_down", "bound": "hbm",
+                      "achieved": ach_s, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": ach_s / peaks["hbm_gbs"], "traffic": None,
+                      "algorithmic_bytes": SHARED_BYTES,
+                      "peak_source": peaks["source"] + " (burst copy)"}
+            bytes_l = uniq * EXPERT_BYTES + SHARED_BYTES
+            ach_l = bytes_l / (ms_l / 1e3) / 1e9
+            roof_l = {"kernel": "whole layer step (router, routed GEMV pair, shared GEMV pair)",
+                      "bound": "hbm", "achieved": ach_l, "peak": peaks["hbm_gbs"],
+                      "unit": "GB/s", "frac": ach_l / peaks["hbm_gbs"], "traffic": None,
+                      "algorithmic_bytes": bytes_l,
+                      "peak_source": peaks["source"] + " (burst copy)"}
+            launches = (2, 5)
+        else:
+            fl_s = 2 * T * 3 * H * SHARED_I
+            ach_s = fl_s / (ms_s / 1e3) / 1e12
+            roof_s = {"kernel": "shared_gemm_kernel (tcgen05, both projections)",
+                      "bound": "tensor", "achieved": ach_s, "peak": peaks["bf16_tflops"],
+                      "unit": "TFLOP/s", "frac": ach_s / peaks["bf16_tflops"], "traffic": None,
+                      "algorithmic_flops": fl_s,
+                      "peak_source": peaks["source"] + " (cuBLAS bf16 burst)"}
+            fl_l = fl_s + 2 * T * K * 3 * H * I
+            ach_l = fl_l / (ms_l / 1e3) / 1e12
+            roof_l = {"kernel": "whole layer step (router, routed tcgen05 GEMMs, shared "
+                                "tcgen05 GEMMs)", "bound": "tensor", "achieved": ach_l,
+                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                      "frac": ach_l / peaks["bf16_tflops"], "traffic": None,
+                      "algorithmic_flops": fl_l,
+                      "peak_source": peaks["source"] + " (cuBLAS bf16 burst)"}
+            launches = (2, 8)
+        common = {"unit": "tokens/s", "higher_is_better": True,
+                  "dtype": "bf16 shared expert (exact products, f32 sums); NVFP4 routed "
+                           "experts", "data": "synthetic"}
+        recs.append({"metric": "shared expert tokens/s", "value": T / (ms_s / 1e3),
+                     "ms_per_step": ms_s, "steps": steps, "warmup": warmup, **common,
+                     "config": {"workload": f"shared expert: H={H} Is={SHARED_I} bf16, T={T}",
+                                "l2": f"{SHARED_COPIES} weight copies rotated "
+                                      f"({SHARED_COPIES * SHARED_BYTES / 1e6:.0f} MB > L2)"},
+                     "roofline": roof_s, "clocks": clk_s, "gpu_launches": launches[0] * steps})
+        recs.append({"metric": METRIC + " (whole layer: router + routed + shared)",
+                     "value": T / (ms_l / 1e3), "ms_per_step": ms_l, "steps": steps,
+                     "warmup": warmup, **common,
+                     "config": {"workload": f"layer: router logits -> top-8 of 256 NVFP4 "
+                                            f"experts + BF16 shared expert (Is={SHARED_I}), "
+                                            f"T={T}" + (", Zipf routing" if T > 1 else ""),
+                                "unique_experts_per_step": uniq,
+                                "l2": "new tokens every step; routed weights 5.4 GB, shared "
+                                      f"weights rotated over {SHARED_COPIES} copies"},
+                     "roofline": roof_l, "clocks": clk_l,
+                     "gpu_launches": launches[1] * steps})
+        del xs, logits, routed, out, sws, lws
+    del shared
+    torch.cuda.empty_cache()
+    return recs
+
+
 SUB_DECODE_STEPS = {"decode1": 4096, "decode8": 1024, "decode32": 512, "decode64": 256}
 
 
 def run_ours(args, rank, world, device):
     import bit_quantized_moe_nvfp4_b200 as nv
     b = Bench(nv, args, rank, world, device)
+    if args.workload == "layer":
+        recs = shared_layer_records(b, args.warmup)
+        return {**recs[-1], "n_gpus": world, "scaling": "weak", "vs_baseline": None,
+                "sub_records": recs}
     if args.workload == "codec":
         rec = b.codec_record(args.steps, args.warmup)
         rec.update({"n_gpus": world, "scaling": "weak", "vs_baseline": None,
@@ -615,6 +745,7 @@ def run_ours(args, rank, world, device):
         subs = []
         for name, n in SUB_DECODE_STEPS.items():
             subs.append(b.layer_record(name, max(n, args.steps), args.warmup, main=False))
+        subs += shared_layer_records(b, args.warmup)
         b.drop_layer()
         subs.append(b.codec_record(max(3, min(args.steps, 8)), args.warmup))
         line["sub_records"] = subs

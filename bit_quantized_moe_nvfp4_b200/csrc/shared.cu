@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kGemvThreads) shared_gemv_down(SharedArgs a) {
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
     for (int c = lane; c < n8; c += 32) {
       const uint4 v = ldg_stream(wd + c);
 #pragma unroll
@@ -175,8 +175,8 @@ constexpr int DS = 4;                           // pipeline stages (64 reduction
 constexpr uint32_t kDA = DBM * 128;             // weight tile per stage: 128 rows x 128 B
 constexpr uint32_t kDB = DBN * 128;             // token tile per stage: 256 rows x 128 B
 constexpr uint32_t kDStage = kDA + kDB;
-constexpr uint32_t kDU = DS * kDStage;          // SwiGLU exchange: 64 up rows x 33 fp32
-constexpr uint32_t kDUBytes = 64 * 33 * 4;
+constexpr uint32_t kDU = DS * kDStage;          // SwiGLU exchange: 64 up rows x 17 fp32
+constexpr uint32_t kDUBytes = 64 * 17 * 4;
 constexpr uint32_t kDBars = kDU + kDUBytes;
 constexpr uint32_t kDMisc = kDBars + 8 * (2 * DS + 4);
 constexpr uint32_t kDSmem = kDMisc + 16 + 1024;   // + alignment slack
@@ -311,37 +311,42 @@ __global__ void __launch_bounds__(kDThreads, 1)
       const int64_t t0 = (int64_t)nt * DBN;
       const int ncols = (int)min64(DBN, T - t0);
       const uint32_t tb = tmem_base + acc * DBN + ((uint32_t)(q * 32) << 16);
-      for (int c0 = 0; c0 < ncols; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tb + c0, v);
+      for (int c0 = 0; c0 < ncols; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tb + c0, v);
         if (p.mode == 0) {
           if (q >= 2) {   // up rows: hand them to the gate rows' threads
 #pragma unroll
-            for (int c = 0; c < 32; ++c) U[(row - 64) * 33 + c] = __uint_as_float(v[c]);
+            for (int c = 0; c < 16; ++c) U[(row - 64) * 17 + c] = __uint_as_float(v[c]);
           }
           named_sync(1, 128);
           if (q < 2) {
             const int64_t j = (int64_t)mt * 64 + row;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < 16; ++c) {
               const int64_t t = t0 + c0 + c;
               if (t < T)
                 a.h[t * Is + j] =
-                    __float2bfloat16_rn(silu_f32(__uint_as_float(v[c])) * U[row * 33 + c]);
+                    __float2bfloat16_rn(silu_f32(__uint_as_float(v[c])) * U[row * 17 + c]);
             }
           }
           named_sync(1, 128);
         } else {
+          // The routed sums of the 16 tokens are all loaded before the first store: the
+          // compiler cannot tell `routed` and `out` apart, so interleaving them would make
+          // every load wait for the store before it.
           const int64_t n = (int64_t)mt * DBM + row;
-          if (n < H) {
+          const bool nv = n < H;
+          float r[16];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int64_t t = t0 + c0 + c;
-              if (t < T) {
-                const float r = a.routed ? __ldcg(a.routed + t * H + n) : 0.f;
-                a.out[t * H + n] = __float2bfloat16_rn(r + __uint_as_float(v[c]));
-              }
-            }
+          for (int c = 0; c < 16; ++c) {
+            const int64_t t = t0 + c0 + c;
+            r[c] = (a.routed && nv && t < T) ? __ldcg(a.routed + t * H + n) : 0.f;
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int64_t t = t0 + c0 + c;
+            if (nv && t < T) a.out[t * H + n] = __float2bfloat16_rn(r[c] + __uint_as_float(v[c]));
           }
         }
       }
