@@ -6,8 +6,10 @@
 //   s = (amax_b / 6) / g  -> E4M3, nearest even, saturating
 //   code_i = E2M1(x_i / (dec(s) * g)), nearest even, saturating, sign kept; 0 if the
 //   divisor is 0.
-// Every step is the IEEE fp32 operation written (no reciprocal, no contraction), so the
-// bits are reproducible.  The kernels stream HBM with 16-byte accesses.
+// The codes and scales are exactly those of the IEEE fp32 operations written (no contraction):
+// the kernels reach them through reciprocal multiplies checked against the rounding
+// boundaries, and divide wherever that check cannot decide (below).  The kernels stream HBM
+// with 16-byte accesses.
 #include "pipeline.cuh"
 
 namespace nvfp4 {
