@@ -76,6 +76,9 @@ def _load():
             L.oracle_nvfp4_dequantize.argtypes = [P, P, P, I64, I64, I64, P]
             L.oracle_route.restype = I64
             L.oracle_route.argtypes = [P, I64, I64, I64, P, P, P, P]
+            L.oracle_moe_forward_w4a4.restype = I64
+            L.oracle_moe_forward_w4a4.argtypes = [P, P, P, I64, I64, I64, I64, I64,
+                                                  P, P, P, P, P, P, P, I64, P, P]
             L.oracle_shared_expert.restype = None
             L.oracle_shared_expert.argtypes = [P, I64, I64, P, P, P, I64, P]
             L.oracle_bf16_round_array.restype = None
@@ -236,12 +239,13 @@ def router(logits, K: int):
 
 
 # ----------------------------------------------------------------------------- MoE
-def moe_forward(x, ids, w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, tokens=None):
+def moe_forward(x, ids, w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, tokens=None, w4a4=False):
     """Routed-expert MoE forward for the listed tokens (all when tokens is None).
 
     x bf16 [T,H]; ids int32 [T,K]; w fp32 [T,K]; w_gu u8 [E,2I,H/2]; s_gu u8 [E,2I,H/16];
     g_gu fp32 [E]; w_dn u8 [E,H,I/2]; s_dn u8 [E,H,I/16]; g_dn fp32 [E].
     Returns (out bf16 bits uint16 [n,H], out fp64 [n,H], number of out-of-range ids).
+    w4a4=True: the activations (x rows, then h rows) are NVFP4-quantized per row as well.
     """
     xs = _u16(x)
     T, H = xs.shape
@@ -257,7 +261,8 @@ def moe_forward(x, ids, w, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn, tokens=None):
     tok = np.arange(T, dtype=np.int64) if tokens is None else _np(tokens, np.int64)
     out = np.zeros((tok.size, H), np.uint16)
     out64 = np.zeros((tok.size, H), np.float64)
-    bad = _load().oracle_moe_forward(_p(xs), _p(ia), _p(wa), T, H, I, E, K,
+    fn = _load().oracle_moe_forward_w4a4 if w4a4 else _load().oracle_moe_forward
+    bad = fn(_p(xs), _p(ia), _p(wa), T, H, I, E, K,
                                      _p(pg), _p(sg), _p(gg), _p(pd), _p(sd), _p(gd),
                                      _p(tok), tok.size, _p(out), _p(out64))
     return out, out64, int(bad)

@@ -468,6 +468,92 @@ int64_t oracle_moe_forward(const uint16_t *x, const int32_t *ids, const float *w
     return bad;
 }
 
+/* One activation row quantized to NVFP4 as a tensor of its own (its own global scale
+ * g = amax(row) / 2688, readings of the codec above) and decoded exactly into v (fp64). */
+static void quantize_row_exact(const uint16_t *row, int64_t n, uint8_t *packed, uint8_t *scales,
+                               double *v)
+{
+    float g;
+    oracle_nvfp4_quantize(row, 1, 1, n, packed, scales, &g);
+    for (int64_t c = 0; c < n; ++c)
+        v[c] = nvfp4_weight(packed, scales, (double)g, n, 0, c);
+}
+
+/* The routed-expert layer with NVFP4 activations as well as NVFP4 weights ("W4A4"), as a
+ * block-scaled FP4 tensor-core GEMM computes it.  Page "GLM-5-NVFP4-MTP", "How to Run",
+ * serves the NVFP4 checkpoint with ModelOpt's FP4 quantization and FP4 MoE kernels.  The
+ * pages do not say how activations are scaled.  [Reading: each activation row, a token's x
+ * for the gate/up projection and a routed pair's bf16 h for the down projection, is
+ * quantized with the codec's readings as a tensor of its own, i.e. with a dynamic
+ * per-row global scale and per-16 block scales.  Its exact NVFP4 values multiply the exact
+ * NVFP4 weights, summed in fp64.  h is rounded to bf16 before it is quantized, as in the
+ * W4A16 forward.]  Arguments, shapes, out-of-range ids and return value as
+ * oracle_moe_forward. */
+int64_t oracle_moe_forward_w4a4(const uint16_t *x, const int32_t *ids, const float *w,
+                                int64_t T, int64_t H, int64_t I, int64_t E, int64_t K,
+                                const uint8_t *wgu, const uint8_t *sgu, const float *ggu,
+                                const uint8_t *wdn, const uint8_t *sdn, const float *gdn,
+                                const int64_t *tok, int64_t n_tok, uint16_t *out, double *out64)
+{
+    (void)T;
+    int64_t bad = 0;
+    int64_t nmax = H > I ? H : I;
+    double *xq = (double *)malloc(sizeof(double) * H);
+    double *a = (double *)malloc(sizeof(double) * 2 * I);
+    uint16_t *hb = (uint16_t *)malloc(sizeof(uint16_t) * I);
+    double *hq = (double *)malloc(sizeof(double) * I);
+    double *acc = (double *)malloc(sizeof(double) * H);
+    uint8_t *pk = (uint8_t *)malloc((size_t)nmax / 2);
+    uint8_t *sc = (uint8_t *)malloc((size_t)nmax / 16);
+    for (int64_t i = 0; i < n_tok; ++i) {
+        int64_t t = tok[i];
+        quantize_row_exact(x + t * H, H, pk, sc, xq);
+        for (int64_t c = 0; c < H; ++c) acc[c] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t e = ids[t * K + k];
+            if (e < 0 || e >= E) {
+                bad++;
+                continue;
+            }
+            const uint8_t *pg = wgu + e * (2 * I) * (H / 2);
+            const uint8_t *sg = sgu + e * (2 * I) * (H / 16);
+            const uint8_t *pd = wdn + e * H * (I / 2);
+            const uint8_t *sd = sdn + e * H * (I / 16);
+            double g1 = ggu[e], g2 = gdn[e];
+            #pragma omp parallel for schedule(static)
+            for (int64_t j = 0; j < 2 * I; ++j) {
+                double s = 0.0;
+                for (int64_t c = 0; c < H; ++c)
+                    s += nvfp4_weight(pg, sg, g1, H, j, c) * xq[c];
+                a[j] = s;
+            }
+            for (int64_t j = 0; j < I; ++j) hb[j] = oracle_bf16_round(silu(a[j]) * a[I + j]);
+            quantize_row_exact(hb, I, pk, sc, hq);
+            double wk = w[t * K + k];
+            #pragma omp parallel for schedule(static)
+            for (int64_t n = 0; n < H; ++n) {
+                double s = 0.0;
+                for (int64_t c = 0; c < I; ++c)
+                    s += nvfp4_weight(pd, sd, g2, I, n, c) * hq[c];
+                acc[n] += wk * s;
+            }
+        }
+        for (int64_t c = 0; c < H; ++c) {
+            out[i * H + c] = oracle_bf16_round(acc[c]);
+            if (out64)
+                out64[i * H + c] = acc[c];
+        }
+    }
+    free(xq);
+    free(a);
+    free(hb);
+    free(hq);
+    free(acc);
+    free(pk);
+    free(sc);
+    return bad;
+}
+
 /* The shared expert: a dense SwiGLU MLP in BF16 that every token passes through, next to
  * the routed experts.  Page "GLM-5-NVFP4-MTP", "What's quantized": only the routed
  * experts' projections are NVFP4 and everything else stays BF16.  A page on the same model

@@ -484,3 +484,61 @@ def test_bf16_round_array_matches_scalar_rounding():
     v = np.concatenate([synth.router_logits(4, 64, seed=1).double().numpy().ravel() * 1e3,
                         [0.0, -0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9, 65504.0]])
     assert [int(b) for b in oracle.bf16_round_array(v)] == [oracle.bf16_round(x) for x in v]
+
+
+# ----------------------------------------------------------------------------- W4A4
+# The layer with NVFP4 activations (reading: each x row and each h row quantized as a tensor
+# of its own), as the block-scaled FP4 tensor-core GEMM computes it.
+
+def _exact_nvfp4(packed, scales, g):
+    """Exact fp64 values of NVFP4 tensors [n, rows, cols/2] + [n, rows, cols/16] + [n]."""
+    e2m1 = np.array([oracle.e2m1_value(c) for c in range(16)])
+    e4m3 = np.array([oracle.e4m3_value(c) if (c & 0x7F) != 0x7F else 0.0 for c in range(256)])
+    lo, hi = packed & 15, packed >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(packed.shape[:-1] + (packed.shape[-1] * 2,))
+    sc = np.repeat(e4m3[scales], 16, axis=-1)
+    return e2m1[codes] * sc * np.asarray(g, np.float64).reshape((-1,) + (1,) * (packed.ndim - 1))
+
+
+def test_w4a4_matches_composition_of_pinned_steps():
+    """Recompose the W4A4 layer from the pinned quantizer, the exact E2M1/E4M3 tables and the
+    pinned bf16 rounding with numpy dense products: quantize each x row, contract with the
+    exact weights, SwiGLU, round h to bf16, quantize each h row, contract, combine."""
+    E, H, I, K, T = 6, 64, 32, 2, 5
+    gu, dn = synth.expert_weights_bf16(E, H, I, seed=8, outlier_p=0.02)
+    pg, sg, gg = oracle.quantize(gu)
+    pd, sd, gd = oracle.quantize(dn)
+    Wg, Wd = _exact_nvfp4(pg, sg, gg), _exact_nvfp4(pd, sd, gd)
+    x = synth.activations_bf16(T, H, 8)
+    ids, w = synth.routing(T, E, K, seed=8)
+    _, out64, bad = oracle.moe_forward(x, ids, w, pg, sg, gg, pd, sd, gd, w4a4=True)
+    assert bad == 0
+    want = np.zeros((T, H))
+    for t in range(T):
+        qp, qs, qg = oracle.quantize(x[t:t + 1].view(1, 1, H))
+        xq = _exact_nvfp4(qp, qs, qg)[0, 0]
+        for k in range(K):
+            e = int(ids[t, k])
+            a = Wg[e] @ xq
+            hh = a[:I] / (1 + np.exp(-a[:I])) * a[I:]
+            hb = torch.from_numpy(oracle.bf16_round_array(hh).astype(np.int16)).view(
+                torch.bfloat16).view(1, 1, I)
+            hp, hs, hg = oracle.quantize(hb)
+            want[t] += float(w[t, k]) * (Wd[e] @ _exact_nvfp4(hp, hs, hg)[0, 0])
+    np.testing.assert_allclose(out64, want, rtol=1e-11, atol=1e-13)
+
+
+def test_w4a4_special_cases():
+    E, H, I, K, T = 4, 64, 32, 2, 3
+    gu, dn = synth.expert_weights_bf16(E, H, I, seed=9)
+    wts = oracle.quantize(gu) + oracle.quantize(dn)
+    ids, w = synth.routing(T, E, K, seed=9)
+    out, out64, _ = oracle.moe_forward(torch.zeros(T, H, dtype=torch.bfloat16), ids, w, *wts,
+                                       w4a4=True)
+    assert np.all(out64 == 0)
+    # quantizing activations moves the output by the NVFP4 noise of x and h, not more
+    x = synth.activations_bf16(T, H, 9)
+    _, a16, _ = oracle.moe_forward(x, ids, w, *wts)
+    _, a4, _ = oracle.moe_forward(x, ids, w, *wts, w4a4=True)
+    rel = np.linalg.norm(a4 - a16) / np.linalg.norm(a16)
+    assert 1e-3 < rel < 0.25
