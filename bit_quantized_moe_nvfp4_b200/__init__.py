@@ -26,6 +26,7 @@ __all__ = [
     "nvfp4_quantize_with_amax", "moe_nvfp4_ep_local_experts", "moe_nvfp4_forward_ep",
     "moe_nvfp4_ep_reduce", "EP_MAX_PARTS", "moe_nvfp4_router", "moe_nvfp4_forward_logits",
     "moe_nvfp4_shared_expert", "moe_nvfp4_layer", "moe_nvfp4_layer_workspace_size",
+    "nvfp4_w4a4_prepare_scales", "moe_nvfp4_forward_w4a4", "moe_nvfp4_w4a4_workspace_size",
 ]
 
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
@@ -72,6 +73,10 @@ def _load() -> ctypes.CDLL:
                                        P, P, P, P, P, P, P, P, SZ, I32, P]),
         "moe_nvfp4_ep_reduce": (I32, [P, I64, I64, I64, P, P]),
         "moe_nvfp4_router": (I32, [P, I64, I64, I64, P, P, P]),
+        "nvfp4_w4a4_prepare_scales": (I32, [P, I64, I64, I64, I64, P, P]),
+        "moe_nvfp4_w4a4_workspace_size": (SZ, [I64, I64, I64, I64, I64]),
+        "moe_nvfp4_forward_w4a4": (I32, [P, P, P, I64, I64, I64, I64, I64,
+                                         P, P, P, P, P, P, P, P, SZ, P]),
         "moe_nvfp4_shared_workspace_size": (SZ, [I64, I64]),
         "moe_nvfp4_shared_expert": (I32, [P, I64, I64, I64, P, P, P, P, P, SZ, P]),
         "moe_nvfp4_layer_workspace_size": (SZ, [I64, I64, I64, I64, I64, I64]),
@@ -378,6 +383,51 @@ def moe_nvfp4_layer(x, router_logits, K: int, w_gu, s_gu, g_gu, w_dn, s_dn, g_dn
         _ptr(w_dn), _ptr(s_dn), _ptr(g_dn), _ptr(shared_gu), _ptr(shared_dn), Is, _ptr(out),
         _ptr(ids_out), _ptr(w_out), _ptr(workspace), workspace.numel(), int(path),
         _stream(x.device)))
+    return out
+
+
+def nvfp4_w4a4_prepare_scales(scales: torch.Tensor, gate_rows: int = 0, out=None):
+    """A weight's E4M3 scales [n, rows, cols/16] rearranged into the block-scaled tensor
+    cores' layout (see include/nvfp4_moe.h); gate_rows = I for a fused gate/up weight."""
+    _need(scales, torch.uint8, "scales")
+    n, rows, c16 = scales.shape
+    if out is None:
+        out = torch.empty_like(scales)
+    _need(out, torch.uint8, "out")
+    _check(_lib().nvfp4_w4a4_prepare_scales(_ptr(scales), n, rows, c16 * 16, int(gate_rows),
+                                            _ptr(out), _stream(scales.device)))
+    return out
+
+
+def moe_nvfp4_w4a4_workspace_size(T, H, I, E, K) -> int:
+    return int(_lib().moe_nvfp4_w4a4_workspace_size(T, H, I, E, K))
+
+
+def moe_nvfp4_forward_w4a4(x, topk_ids, topk_w, w_gu, sf_gu, g_gu, w_dn, sf_dn, g_dn,
+                           out=None, workspace=None) -> torch.Tensor:
+    """The routed layer on the FP4 tensor cores with NVFP4 activations (W4A4); sf_gu / sf_dn
+    are the prepared scales.  Returns out bf16 [T, H]."""
+    _need(x, torch.bfloat16, "x")
+    _need(topk_ids, torch.int32, "topk_ids")
+    _need(topk_w, torch.float32, "topk_w")
+    for t, n in ((w_gu, "w_gu"), (sf_gu, "sf_gu"), (w_dn, "w_dn"), (sf_dn, "sf_dn")):
+        _need(t, torch.uint8, n)
+    _need(g_gu, torch.float32, "g_gu")
+    _need(g_dn, torch.float32, "g_dn")
+    T, H = x.shape
+    K = topk_ids.shape[1]
+    E, twoI, _ = w_gu.shape
+    I = twoI // 2
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((moe_nvfp4_w4a4_workspace_size(T, H, I, E, K),),
+                                dtype=torch.uint8, device=x.device)
+        workspace[:WORKSPACE_ZERO_BYTES].zero_()
+    _check(_lib().moe_nvfp4_forward_w4a4(
+        _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, I, E, K, _ptr(w_gu), _ptr(sf_gu),
+        _ptr(g_gu), _ptr(w_dn), _ptr(sf_dn), _ptr(g_dn), _ptr(out), _ptr(workspace),
+        workspace.numel(), _stream(x.device)))
     return out
 
 

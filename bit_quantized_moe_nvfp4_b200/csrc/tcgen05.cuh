@@ -33,6 +33,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
+// Shared-memory matrix descriptor, no swizzle, K-major, for 16-byte rows stored one after
+// another (8-row core matrices of 128 contiguous bytes): the source of a tcgen05.cp of
+// 32 rows x 128 bits.
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);   // start address, 16-byte units
+  d |= (uint64_t)(128 >> 4) << 16;           // leading byte offset (one core matrix along K)
+  d |= (uint64_t)(128 >> 4) << 32;           // stride byte offset: 8 rows * 16 B
+  d |= (uint64_t)1 << 46;                    // descriptor version (sm_100); layout 0: none
+  return d;
+}
+
+// Instruction descriptor of kind::mxf4nvf4 (block-scaled): E2M1 A and B (both K-major), one
+// UE4M3 scale per 16 elements along K, fp32 D, K = 64 per instruction; scale factors at byte
+// 0 of their tensor-memory words.
+__host__ __device__ constexpr uint32_t idesc_nvfp4_f32(int M, int N) {
+  return (1u << 7)                      // A format: E2M1
+         | (1u << 10)                   // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16  (scale format bit 23 = 0: UE4M3; K64)
+}
+
 // Instruction descriptor of kind::f16 with f16 A and B, fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4)                      // D format: f32 (A, B format 0: f16)
@@ -61,6 +83,30 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
       : "memory");
+}
+
+// D[tmem] (+)= (A . SFA)[smem] * (B . SFB)[smem]^T for NVFP4 operands: M x N x 64, the scale
+// factors of A and B read from tensor memory (one 32-bit word per row: its four UE4M3
+// scales of the 64-element K slice).  Issued by one thread.
+__device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                           bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;"
+      "\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate),
+        "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory (descriptor) to tensor memory at `taddr`,
+// repeated into each of the four 32-lane quarters.  Issued by one thread; ordered with the
+// thread's later tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread is done.

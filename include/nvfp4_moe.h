@@ -341,6 +341,45 @@ NVFP4_API int moe_nvfp4_forward_ep(const __nv_bfloat16 *x, const int32_t *topk_i
 NVFP4_API int moe_nvfp4_ep_reduce(const float *const *partials, int64_t n_parts, int64_t rows,
                                   int64_t cols, __nv_bfloat16 *out, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- W4A4 (FP4 tensor cores) */
+
+/* The routed layer on the block-scaled FP4 tensor cores (tcgen05.mma kind::mxf4nvf4).  Page
+ * "GLM-5-NVFP4-MTP", "How to Run", serves the NVFP4 checkpoint with ModelOpt FP4 quantization
+ * and FP4 MoE kernels.  The activations are quantized to NVFP4 on the fly.  Each activation
+ * row (a token's x for gate/up, a routed pair's bf16 h for down) is quantized as a tensor of
+ * its own: global scale amax(row) / 2688, E4M3 scale per 16, E2M1 codes, exactly as
+ * nvfp4_quantize.  Its exact NVFP4 values multiply the exact NVFP4 weights with fp32
+ * accumulation.  This computes a different function from moe_nvfp4_forward, whose
+ * activations stay bf16; the pages fix no activation format.
+ *
+ * The tensor cores take block scales in their own layout.  nvfp4_w4a4_prepare_scales
+ * rearranges a weight tensor's E4M3 scales ([n, rows, cols/16], as nvfp4_quantize writes
+ * them) into it, once per weight: one 512-byte atom per 128 rows and 64 columns, row r's four
+ * scales in the 32-bit word at byte 16 (r % 32) + 4 (r / 32).  gate_rows = I for a fused
+ * gate/up weight [2I, cols], whose atom group m then holds gate rows 64m.. and up rows
+ * I + 64m..; gate_rows = 0 for a plain weight (group m = rows 128m..).  out has the size of
+ * scales.  Limits: rows % 128 == 0, cols % 64 == 0; 4-byte aligned pointers.
+ * Errors: EINVAL, ESHAPE, ECUDA. */
+NVFP4_API int nvfp4_w4a4_prepare_scales(const uint8_t *scales, int64_t n_tensors, int64_t rows,
+                                        int64_t cols, int64_t gate_rows, uint8_t *out,
+                                        cudaStream_t stream);
+
+/* The W4A4 forward.  Arguments as moe_nvfp4_forward, except that sf_gu / sf_dn are the
+ * prepared scales (nvfp4_w4a4_prepare_scales with gate_rows I, resp. 0).  Runs the
+ * tensor-core path for any T.  Limits: H % 256 == 0, I % 256 == 0, K <= 16, E <= 1024.
+ * Workspace: moe_nvfp4_w4a4_workspace_size bytes, first NVFP4_WORKSPACE_ZERO_BYTES zero
+ * before first use (the error flag is its first word, as for moe_nvfp4_forward).
+ * Errors: EINVAL, ESHAPE, EWORKSPACE, ECUDA. */
+NVFP4_API size_t moe_nvfp4_w4a4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E,
+                                               int64_t K);
+NVFP4_API int moe_nvfp4_forward_w4a4(const __nv_bfloat16 *x, const int32_t *topk_ids,
+                                     const float *topk_w, int64_t T, int64_t H, int64_t I,
+                                     int64_t E, int64_t K, const uint8_t *w_gu,
+                                     const uint8_t *sf_gu, const float *g_gu,
+                                     const uint8_t *w_dn, const uint8_t *sf_dn,
+                                     const float *g_dn, __nv_bfloat16 *out, void *workspace,
+                                     size_t ws_bytes, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- fixed-scratch forward */
 
 /* Bytes of the fixed scratch of moe_nvfp4_forward_static: it holds 256 bytes of counters,

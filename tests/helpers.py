@@ -110,7 +110,7 @@ class FullLayer:
         return [np.stack([p[i] for p in per]) for i in range(6)]
 
 
-def check_sampled(full, x, ids, w, out, tokens, ep=None):
+def check_sampled(full, x, ids, w, out, tokens, ep=None, w4a4=False):
     """Compare the listed tokens of `out` with the oracle, token by token, in one oracle call
     over the union of their experts.  ep=(G, r): `out` is rank r's fp32 partial of an
     expert-parallel forward over G ranks, compared with the oracle's sum over that rank's
@@ -121,7 +121,7 @@ def check_sampled(full, x, ids, w, out, tokens, ep=None):
     ids_s = torch.tensor([[remap[int(e)] for e in ids[t]] for t in tokens], dtype=torch.int32)
     host = full.oracle_inputs(experts)
     w_s = w[tokens] if ep is None else owned_weights(ids[tokens], w[tokens], full.E, *ep)
-    ref, ref64, bad = oracle.moe_forward(x[tokens], ids_s, w_s, *host)
+    ref, ref64, bad = oracle.moe_forward(x[tokens], ids_s, w_s, *host, w4a4=w4a4)
     assert bad == 0
     for n, t in enumerate(tokens):
         if ep is None:

@@ -220,6 +220,39 @@ def test_router_argument_checks_run_before_cuda(lib):
     assert call(ws_bytes=16) == -3
 
 
+def test_w4a4_argument_checks_run_before_cuda(lib):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    fake = ctypes.c_void_p(1 << 20)
+    pr = lib.nvfp4_w4a4_prepare_scales
+    pr.restype = ctypes.c_int
+    pr.argtypes = [P, I64, I64, I64, I64, P, P]
+    assert pr(None, 1, 128, 64, 0, fake, None) == -1
+    assert pr(fake, 1, 100, 64, 0, fake, None) == -2       # rows % 128
+    assert pr(fake, 1, 128, 48, 0, fake, None) == -2       # cols % 64
+    assert pr(fake, 1, 256, 64, 64, fake, None) == -2      # gate rows must be half the rows
+    assert pr(ctypes.c_void_p((1 << 20) + 2), 1, 128, 64, 0, fake, None) == -1
+    f = lib.moe_nvfp4_forward_w4a4
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, I64, I64, I64, I64, I64, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+
+    def call(ptr=fake, ws_bytes=1 << 40, **over):
+        d = dict(dict(T=4, H=6144, I=2048, E=256, K=8), **over)
+        return f(ptr, ptr, ptr, d["T"], d["H"], d["I"], d["E"], d["K"], ptr, ptr, ptr, ptr,
+                 ptr, ptr, ptr, fake, ws_bytes, None)
+
+    assert call(ptr=None) == -1
+    assert call(H=6208) == -2                               # H % 256
+    assert call(I=2112) == -2                               # I % 256
+    assert call(K=17) == -2
+    assert call(ws_bytes=16) == -3
+    ws = lib.moe_nvfp4_w4a4_workspace_size
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [I64] * 5
+    lib.moe_nvfp4_workspace_size.restype = ctypes.c_size_t
+    lib.moe_nvfp4_workspace_size.argtypes = [I64] * 5
+    assert ws(4096, 6144, 2048, 256, 8) > lib.moe_nvfp4_workspace_size(4096, 6144, 2048, 256, 8)
+
+
 def test_selftest_argument_checks_run_before_cuda(lib):
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     f = lib.nvfp4_selftest_wait_timeout
