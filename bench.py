@@ -2,7 +2,7 @@
 """Benchmark of the NVFP4 routed-expert MoE layer on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload all|prefill|decode1|decode8|decode32|decode64|codec|layer]
+                    [--workload all|prefill|decode1|decode8|decode32|decode64|codec|layer|w4a4]
 
 A step is one pass of the whole layer (route -> gate/up + SwiGLU -> down -> combine) over
 one batch of the H=6144, I=2048, E=256, top-8 layer whose NVFP4 weights (5.4 GB, N(0,0.02)
@@ -13,8 +13,10 @@ a NEW batch, so the expert bytes it reads are not left in the 126 MB L2 by the s
 Steps are replayed from a CUDA graph and timed with CUDA events on the launching stream.
 
 With --workload all (the default, one GPU) the line also carries `sub_records`: decode of
-T = 1, 8, 32 and 64 tokens (HBM-bound GEMV path) and the whole-layer quantize / dequantize
-sweep, each timed the same way with its own step count, clock samples and roofline.
+T = 1, 8, 32 and 64 tokens (HBM-bound GEMV path), the BF16 shared expert and the whole layer
+(router + routed + shared) at T = 1 and 4096, the prefill batch on the FP4 tensor cores
+(W4A4), and the whole-layer codec legs, each timed the same way with its own step count,
+clock samples and roofline.
 
 Keys beyond the base contract: `roofline` (dominant kernel; live CUDA-event durations of
 each stage from a second, marked pass), `cpu_baseline` (the CPU oracle on a bounded
@@ -720,12 +722,76 @@ def shared_layer_records(b, warmup):
     return recs
 
 
+FP4_PER_BF16 = 4.0   # nominal dense FP4 : bf16 tensor-core rate (9 : 2.25 PFLOP/s)
+
+
+def w4a4_record(b, steps, warmup):
+    """The prefill batch on the block-scaled FP4 tensor cores (W4A4: NVFP4 activations)."""
+    nv, device, peaks, world = b.nv, b.device, b.peaks, b.world
+    wl = synth.PREFILL_T4096
+    T = wl.T
+    layer = b.ensure_layer()
+    w_gu, s_gu, g_gu, w_dn, s_dn, g_dn = layer
+    prep = (w_gu, nv.nvfp4_w4a4_prepare_scales(s_gu, gate_rows=I), g_gu,
+            w_dn, nv.nvfp4_w4a4_prepare_scales(s_dn), g_dn)
+    n_b = 2
+    xs, ids, ws_ = make_batches(wl, n_b, seed=1000 + b.rank, device=device)
+    ws = torch.zeros((nv.moe_nvfp4_w4a4_workspace_size(T, H, I, E, K),), dtype=torch.uint8,
+                     device=device)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.Stream(device)
+
+    def step(i):
+        nv.moe_nvfp4_forward_w4a4(xs[i], ids[i], ws_[i], *prep, out=out, workspace=ws)
+
+    ms, clk = graph_timed(stream, step, n_b, steps, warmup)
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_b)]
+    for m in marks:
+        for e in m:
+            e.record()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(n_b):
+            nv.moe_nvfp4_forward_w4a4_profiled(xs[i], ids[i], ws_[i], *prep, out, ws, marks[i])
+    torch.cuda.synchronize()
+    names = ["route_quantize_x", "gate_up", "quantize_h_down", "combine"]
+    stages = {n: statistics.mean(m[j].elapsed_time(m[j + 1]) for m in marks)
+              for j, n in enumerate(names)}
+    fl_gu = 2 * T * K * (2 * I * H)
+    pk = peaks["bf16_tflops"] * FP4_PER_BF16
+    ach = fl_gu / (stages["gate_up"] / 1e3) / 1e12
+    flops_step = 2 * T * K * (3 * H * I)
+    rec = {"metric": METRIC + " (W4A4: NVFP4 activations, FP4 tensor cores)",
+           "value": T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "warmup": warmup, "higher_is_better": True,
+           "dtype": "e2m1 x e2m1 products with e4m3 block scales (tcgen05 kind::mxf4nvf4), f32 "
+                    "accumulation",
+           "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) bf16 weights quantized to NVFP4)",
+           "config": {"workload": wl.name + ", W4A4 (each activation row quantized to NVFP4)",
+                      "T": T, "H": H, "I": I, "E": E, "K": K,
+                      "l2": "new tokens every step over 5.4 GB of resident weights",
+                      "timing": f"CUDA graph of {n_b} steps replayed, CUDA events"},
+           "stages_ms": stages, "tflops_step": flops_step / (ms / 1e3) / 1e12,
+           "roofline": {"kernel": "w4a4_gemm_kernel mode 0 (block-scaled FP4 MMA + SwiGLU)",
+                        "bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+                        "frac": ach / pk, "traffic": None, "algorithmic_flops": fl_gu,
+                        "peak_source": peaks["source"] + " (cuBLAS bf16 burst x 4, the "
+                                                         "nominal dense FP4:bf16 ratio)"},
+           "clocks": clk, "gpu_launches": 6 * steps}
+    del prep, xs, ids, ws_, ws, out
+    torch.cuda.empty_cache()
+    return rec
+
+
 SUB_DECODE_STEPS = {"decode1": 4096, "decode8": 1024, "decode32": 512, "decode64": 256}
 
 
 def run_ours(args, rank, world, device):
     import bit_quantized_moe_nvfp4_b200 as nv
     b = Bench(nv, args, rank, world, device)
+    if args.workload == "w4a4":
+        rec = w4a4_record(b, args.steps, args.warmup)
+        return {**rec, "n_gpus": world, "scaling": "weak", "vs_baseline": None}
     if args.workload == "layer":
         recs = shared_layer_records(b, args.warmup)
         return {**recs[-1], "n_gpus": world, "scaling": "weak", "vs_baseline": None,
@@ -746,6 +812,7 @@ def run_ours(args, rank, world, device):
         for name, n in SUB_DECODE_STEPS.items():
             subs.append(b.layer_record(name, max(n, args.steps), args.warmup, main=False))
         subs += shared_layer_records(b, args.warmup)
+        subs.append(w4a4_record(b, max(args.steps, 10), args.warmup))
         b.drop_layer()
         subs.append(b.codec_record(max(3, min(args.steps, 8)), args.warmup))
         line["sub_records"] = subs

@@ -75,6 +75,8 @@ def _load() -> ctypes.CDLL:
         "moe_nvfp4_router": (I32, [P, I64, I64, I64, P, P, P]),
         "nvfp4_w4a4_prepare_scales": (I32, [P, I64, I64, I64, I64, P, P]),
         "moe_nvfp4_w4a4_workspace_size": (SZ, [I64, I64, I64, I64, I64]),
+        "moe_nvfp4_forward_w4a4_profiled": (I32, [P, P, P, I64, I64, I64, I64, I64,
+                                                  P, P, P, P, P, P, P, P, SZ, P, P]),
         "moe_nvfp4_forward_w4a4": (I32, [P, P, P, I64, I64, I64, I64, I64,
                                          P, P, P, P, P, P, P, P, SZ, P]),
         "moe_nvfp4_shared_workspace_size": (SZ, [I64, I64]),
@@ -428,6 +430,20 @@ def moe_nvfp4_forward_w4a4(x, topk_ids, topk_w, w_gu, sf_gu, g_gu, w_dn, sf_dn, 
         _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, I, E, K, _ptr(w_gu), _ptr(sf_gu),
         _ptr(g_gu), _ptr(w_dn), _ptr(sf_dn), _ptr(g_dn), _ptr(out), _ptr(workspace),
         workspace.numel(), _stream(x.device)))
+    return out
+
+
+def moe_nvfp4_forward_w4a4_profiled(x, topk_ids, topk_w, w_gu, sf_gu, g_gu, w_dn, sf_dn, g_dn,
+                                    out, workspace, stage_events):
+    """moe_nvfp4_forward_w4a4 with five torch.cuda.Event recorded between its stages."""
+    T, H = x.shape
+    K = topk_ids.shape[1]
+    E, twoI, _ = w_gu.shape
+    arr = (ctypes.c_void_p * 5)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
+    _check(_lib().moe_nvfp4_forward_w4a4_profiled(
+        _ptr(x), _ptr(topk_ids), _ptr(topk_w), T, H, twoI // 2, E, K, _ptr(w_gu), _ptr(sf_gu),
+        _ptr(g_gu), _ptr(w_dn), _ptr(sf_dn), _ptr(g_dn), _ptr(out), _ptr(workspace),
+        workspace.numel(), arr, _stream(x.device)))
     return out
 
 

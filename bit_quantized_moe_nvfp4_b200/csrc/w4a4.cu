@@ -416,7 +416,29 @@ int launch_w4a4_gemm(const W4Gemm &p, const uint8_t *wq, int64_t w_rows, const u
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// A timing mark between two kernels (external event under stream capture).
+int mark(cudaEvent_t const *ev, int i, cudaStream_t s) {
+  if (!ev) return NVFP4_OK;
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &st);
+  if (e == cudaSuccess)
+    e = st == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev[i], s, cudaEventRecordExternal)
+                                            : cudaEventRecord(ev[i], s);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return NVFP4_ECUDA;
+  }
+  return NVFP4_OK;
+}
+
 }  // namespace
+
+// The W4A4 forward, with timing marks between the stages when ev is not null.
+int forward_w4a4(const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w, int64_t T,
+                 int64_t H, int64_t I, int64_t E, int64_t K, const uint8_t *w_gu,
+                 const uint8_t *sf_gu, const float *g_gu, const uint8_t *w_dn,
+                 const uint8_t *sf_dn, const float *g_dn, __nv_bfloat16 *out, void *workspace,
+                 size_t ws_bytes, cudaEvent_t const *ev, cudaStream_t stream);
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -450,6 +472,29 @@ extern "C" int moe_nvfp4_forward_w4a4(const __nv_bfloat16 *x, const int32_t *top
                                       const uint8_t *w_dn, const uint8_t *sf_dn,
                                       const float *g_dn, __nv_bfloat16 *out, void *workspace,
                                       size_t ws_bytes, cudaStream_t stream) {
+  return forward_w4a4(x, topk_ids, topk_w, T, H, I, E, K, w_gu, sf_gu, g_gu, w_dn, sf_dn, g_dn,
+                      out, workspace, ws_bytes, nullptr, stream);
+}
+
+extern "C" int moe_nvfp4_forward_w4a4_profiled(
+    const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w, int64_t T, int64_t H,
+    int64_t I, int64_t E, int64_t K, const uint8_t *w_gu, const uint8_t *sf_gu, const float *g_gu,
+    const uint8_t *w_dn, const uint8_t *sf_dn, const float *g_dn, __nv_bfloat16 *out,
+    void *workspace, size_t ws_bytes, void *const *stage_events, cudaStream_t stream) {
+  if (!stage_events) return NVFP4_EINVAL;
+  for (int i = 0; i < 5; ++i)
+    if (!stage_events[i]) return NVFP4_EINVAL;
+  return forward_w4a4(x, topk_ids, topk_w, T, H, I, E, K, w_gu, sf_gu, g_gu, w_dn, sf_dn, g_dn,
+                      out, workspace, ws_bytes,
+                      reinterpret_cast<cudaEvent_t const *>(stage_events), stream);
+}
+
+int nvfp4::forward_w4a4(const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w,
+                        int64_t T, int64_t H, int64_t I, int64_t E, int64_t K,
+                        const uint8_t *w_gu, const uint8_t *sf_gu, const float *g_gu,
+                        const uint8_t *w_dn, const uint8_t *sf_dn, const float *g_dn,
+                        __nv_bfloat16 *out, void *workspace, size_t ws_bytes,
+                        cudaEvent_t const *ev, cudaStream_t stream) {
   if (!x || !topk_ids || !topk_w || !w_gu || !sf_gu || !g_gu || !w_dn || !sf_dn || !g_dn || !out)
     return NVFP4_EINVAL;
   if (T <= 0 || H <= 0 || I <= 0 || E <= 0 || K <= 0) return NVFP4_EINVAL;
@@ -501,6 +546,7 @@ extern "C" int moe_nvfp4_forward_w4a4(const __nv_bfloat16 *x, const int32_t *top
   r.n_active = a.n_active;
   r.tile_prefix = a.tile_prefix;
   r.tile_n = kPadN;
+  if (int s = mark(ev, 0, stream)) return s;
   if (int s = launch_route(r, stream, true)) return s;
 
   const Tables tb = {a.counts, a.offsets, a.active, a.n_active, a.tile_prefix, a.perm};
@@ -508,6 +554,7 @@ extern "C" int moe_nvfp4_forward_w4a4(const __nv_bfloat16 *x, const int32_t *top
   uint8_t *hq = reinterpret_cast<uint8_t *>(ws + W.hq), *hsf = reinterpret_cast<uint8_t *>(ws + W.hsf);
   float *gx = reinterpret_cast<float *>(ws + W.gx), *gh = reinterpret_cast<float *>(ws + W.gh);
   if (int s = launch_quant_rows(0, tb, x, H, K, W.P, xq, xsf, gx, stream)) return s;
+  if (int s = mark(ev, 1, stream)) return s;
 
   W4Gemm g = {};
   g.tb = tb;
@@ -525,6 +572,7 @@ extern "C" int moe_nvfp4_forward_w4a4(const __nv_bfloat16 *x, const int32_t *top
   g.g_act = gx;
   g.h = a.h;
   if (int s = launch_w4a4_gemm(g, w_gu, E * 2 * I, xq, W.P, stream)) return s;
+  if (int s = mark(ev, 2, stream)) return s;
 
   if (int s = launch_quant_rows(1, tb, a.h, I, K, W.P, hq, hsf, gh, stream)) return s;
 
@@ -538,5 +586,7 @@ extern "C" int moe_nvfp4_forward_w4a4(const __nv_bfloat16 *x, const int32_t *top
   g.g_act = gh;
   g.y = a.y;
   if (int s = launch_w4a4_gemm(g, w_dn, E * H, hq, W.P, stream)) return s;
-  return launch_combine(a, stream);
+  if (int s = mark(ev, 3, stream)) return s;
+  if (int s = launch_combine(a, stream)) return s;
+  return mark(ev, 4, stream);
 }

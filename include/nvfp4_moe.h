@@ -380,6 +380,16 @@ NVFP4_API int moe_nvfp4_forward_w4a4(const __nv_bfloat16 *x, const int32_t *topk
                                      const float *g_dn, __nv_bfloat16 *out, void *workspace,
                                      size_t ws_bytes, cudaStream_t stream);
 
+/* moe_nvfp4_forward_w4a4 with timing marks: five caller events recorded on `stream` before
+ * the route step, after the x quantization, after the gate/up GEMM, after the h quantization
+ * and down GEMM, and after the combine.  Errors as moe_nvfp4_forward_w4a4, plus EINVAL for a
+ * null event. */
+NVFP4_API int moe_nvfp4_forward_w4a4_profiled(
+    const __nv_bfloat16 *x, const int32_t *topk_ids, const float *topk_w, int64_t T, int64_t H,
+    int64_t I, int64_t E, int64_t K, const uint8_t *w_gu, const uint8_t *sf_gu, const float *g_gu,
+    const uint8_t *w_dn, const uint8_t *sf_dn, const float *g_dn, __nv_bfloat16 *out,
+    void *workspace, size_t ws_bytes, void *const *stage_events, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- fixed-scratch forward */
 
 /* Bytes of the fixed scratch of moe_nvfp4_forward_static: it holds 256 bytes of counters,
