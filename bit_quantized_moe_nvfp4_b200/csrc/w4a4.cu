@@ -38,6 +38,10 @@ namespace {
 
 constexpr int kPadN = 128;   // slots per n-tile (MMA N <= 128)
 
+// silu(z) = z / (1 + e^-z) with the fast exponential and division (a few ulp of fp32; h is
+// rounded to bf16 right after).  For z below about -88, e^-z is infinite and the quotient 0.
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
 __host__ __device__ __forceinline__ int64_t round_up(int64_t v, int64_t m) {
   return (v + m - 1) / m * m;
 }
@@ -150,9 +154,13 @@ constexpr uint32_t kQA = 128 * 128;              // weight tile: 128 rows x 128 
 constexpr uint32_t kQB = kPadN * 128;            // activation tile: 128 slots x 128 bytes
 constexpr uint32_t kQSF = 4 * 512;               // four scale atoms (256 elements of K)
 constexpr uint32_t kQStage = kQA + kQB + 2 * kQSF;
-constexpr uint32_t kQU = QS * kQStage;           // SwiGLU exchange: 64 up rows x 17 fp32
-constexpr uint32_t kQUBytes = 64 * 17 * 4;
-constexpr uint32_t kQBars = kQU + kQUBytes;
+// Epilogue scratch: the 16-slot chunk staged for coalesced stores (down: 16 x 132 fp32;
+// gate/up: the exchanged gate and up halves, 2 x 64 x 9 fp32, then 16 x 64 bf16 of h), and
+// the tile's per-slot factors (128 fp32).
+constexpr uint32_t kQE = QS * kQStage;
+constexpr uint32_t kQEBytes = 16 * 132 * 4;
+constexpr uint32_t kQCol = kQE + kQEBytes;
+constexpr uint32_t kQBars = kQCol + kPadN * 4;
 constexpr uint32_t kQMisc = kQBars + 8 * (2 * QS + 4);
 constexpr uint32_t kQSmem = kQMisc + 16 + 1024;  // + alignment slack
 constexpr int kQThreads = 192;                   // producer, MMA, 4 epilogue warps
@@ -189,7 +197,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint64_t *accempty = accfull + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kQMisc);
   int *abort = reinterpret_cast<int *>(smem + kQMisc + 4);
-  float *U = reinterpret_cast<float *>(smem + kQU);
+  float *ebuf = reinterpret_cast<float *>(smem + kQE);
+  float *colf = reinterpret_cast<float *>(smem + kQCol);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -304,8 +313,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue (warps 2-5)
+    // Warp w reads TMEM lanes 32 (w % 4) .. +31: lane L is weight row L of the tile.  A chunk
+    // of 16 slots leaves through shared memory, so every global store is a 16-byte piece of
+    // one slot's row.
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;   // 0..127
     int tc = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
       int e, mt, nvalid;
@@ -314,40 +327,63 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const int acc = tc & 1;
       if (!wait(&accfull[acc], (tc >> 1) & 1)) break;
       tc_fence_after();
-      const float gw = __ldg(p.g_w + e);
+      {   // the slot's factor: g_w * g_row, times the routing weight for down
+        float f = 0.f;
+        if (et < nvalid) {
+          f = __ldg(p.g_w + e) * __ldg(p.g_act + pad0 + et);
+          if (p.mode == 1) f *= __ldg(p.w + __ldg(p.tb.perm + slot0 + et));
+        }
+        colf[et] = f;
+      }
+      named_sync(1, 128);
       const uint32_t tbase = tmem_base + acc * kPadN + ((uint32_t)(q * 32) << 16);
       for (int c0 = 0; c0 < nvalid; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tbase + c0, v);
-        // per-column factors, all loaded before any store of this chunk
-        float f[16];
+        float val[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const bool cv = c0 + c < nvalid;
-          float fc = cv ? gw * __ldg(p.g_act + pad0 + c0 + c) : 0.f;
-          if (p.mode == 1 && cv) fc *= __ldg(p.w + __ldg(p.tb.perm + slot0 + c0 + c));
-          f[c] = fc;
-        }
+        for (int c = 0; c < 16; ++c) val[c] = __uint_as_float(v[c]) * colf[c0 + c];
         if (p.mode == 0) {
-          if (q >= 2) {   // up rows: hand them to the gate rows' threads
+          // gate rows (lanes 0-63) keep columns 0-7 and hand over 8-15; up rows the reverse
+          float *G = ebuf, *U = ebuf + 64 * 9;
+          __nv_bfloat16 *hs = reinterpret_cast<__nv_bfloat16 *>(ebuf + 128 * 9);   // [16][64]
+          if (q < 2) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) U[(row - 64) * 17 + c] = __uint_as_float(v[c]) * f[c];
+            for (int c = 0; c < 8; ++c) G[row * 9 + c] = val[8 + c];
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) U[(row - 64) * 9 + c] = val[c];
           }
           named_sync(1, 128);
           if (q < 2) {
-            const int64_t j = (int64_t)mt * 64 + row;
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              if (c0 + c < nvalid)
-                p.h[(slot0 + c0 + c) * I + j] =
-                    __float2bfloat16_rn(silu_f32(__uint_as_float(v[c]) * f[c]) * U[row * 17 + c]);
+            for (int c = 0; c < 8; ++c)
+              hs[c * 64 + row] = __float2bfloat16_rn(silu_fast(val[c]) * U[row * 9 + c]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              hs[(8 + c) * 64 + row - 64] =
+                  __float2bfloat16_rn(silu_fast(G[(row - 64) * 9 + c]) * val[8 + c]);
           }
           named_sync(1, 128);
+          const int c = et >> 3, part = et & 7;   // 16 slots x 8 pieces of 16 bytes
+          if (c0 + c < nvalid)
+            *reinterpret_cast<uint4 *>(p.h + (slot0 + c0 + c) * I + mt * 64 + part * 8) =
+                *reinterpret_cast<const uint4 *>(hs + c * 64 + part * 8);
+          named_sync(1, 128);
         } else {
-          const int64_t n = (int64_t)mt * 128 + row;
+          float *ys = ebuf;   // [16][132]
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            if (c0 + c < nvalid) p.y[(slot0 + c0 + c) * H + n] = __uint_as_float(v[c]) * f[c];
+          for (int c = 0; c < 16; ++c) ys[c * 132 + row] = val[c];
+          named_sync(1, 128);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {   // 16 slots x 32 pieces of 16 bytes
+            const int pi = et + 128 * k, c = pi >> 5, part = pi & 31;
+            if (c0 + c < nvalid)
+              *reinterpret_cast<float4 *>(p.y + (slot0 + c0 + c) * H + mt * 128 + part * 4) =
+                  *reinterpret_cast<const float4 *>(ys + c * 132 + part * 4);
+          }
+          named_sync(1, 128);
         }
       }
       tc_fence_before();
