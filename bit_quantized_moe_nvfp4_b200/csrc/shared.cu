@@ -12,8 +12,9 @@
 //
 // Two implementations of one function:
 //  * T <= kGemvMaxT tokens: the 3 * Is * H weights are the whole cost (75 MB at H = 6144,
-//    Is = 2048).  Each warp streams whole weight rows with 16-byte loads against the tokens
-//    held in shared memory and reduces across its lanes; one wave of CTAs covers the rows.
+//    Is = 2048).  Warps stream weight rows with 16-byte loads against the tokens held in
+//    shared memory (gate/up: four warps per row pair, down: one per row) and reduce across
+//    their lanes.
 //  * more tokens: one tcgen05 GEMM per projection.  A CTA tile is 128 weight rows (gate/up:
 //    64 gate rows and the matching 64 up rows, so the SwiGLU stays inside the tile) by 256
 //    tokens.  Both operands come by TMA into a 4-stage ring of 128-byte-swizzled shared
@@ -63,50 +64,71 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ------------------------------------------------------------------ few tokens (CUDA cores)
-// Gate/up: warp w of the grid takes row pairs j = w, w + warps, ...; the tokens' x rows sit
-// in shared memory.  Lane t < T writes h[t, j].
+// Gate/up: the reduction of each row pair (gate row j, up row Is + j) is split over kSplit
+// warps of one CTA, so a CTA of 8 warps takes 8 / kSplit row pairs per pass and every SM
+// holds enough loads in flight; the tokens' x rows sit in shared memory.  The kSplit partial
+// sums are added in warp order, then lane t < T of the finishing threads writes h[t, j].
+constexpr int kSplit = 4;
 template <int NT>
 __global__ void __launch_bounds__(kGemvThreads) shared_gemv_gateup(SharedArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int kRowPairs = kGemvThreads / 32 / kSplit;   // row pairs per CTA pass
+  __shared__ float part_sum[kRowPairs][kSplit][NT][2];
   uint4 *xs = reinterpret_cast<uint4 *>(smem);   // [T][H / 8]
   const int T = (int)a.T;
   const int64_t H = a.H, Is = a.Is;
   const int n8 = (int)(H / 8);
+  const int per = n8 / kSplit;                   // 16-byte words of a row per warp
   pdl_wait();   // x may come from the previous kernel
   for (int i = threadIdx.x; i < T * n8; i += blockDim.x)
     xs[i] = __ldg(reinterpret_cast<const uint4 *>(a.x) + i);
   __syncthreads();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t j = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp; j < Is; j += nwarps) {
-    const uint4 *wg = reinterpret_cast<const uint4 *>(a.w_gu + j * H);
-    const uint4 *wu = reinterpret_cast<const uint4 *>(a.w_gu + (Is + j) * H);
+  const int rp = warp / kSplit, part = warp % kSplit;
+  for (int64_t j0 = (int64_t)blockIdx.x * kRowPairs; j0 < Is; j0 += (int64_t)gridDim.x * kRowPairs) {
+    const int64_t j = j0 + rp;
     float g[NT], u[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) g[t] = u[t] = 0.f;
+    if (j < Is) {
+      const uint4 *wg = reinterpret_cast<const uint4 *>(a.w_gu + j * H);
+      const uint4 *wu = reinterpret_cast<const uint4 *>(a.w_gu + (Is + j) * H);
 #pragma unroll 4
-    for (int c = lane; c < n8; c += 32) {
-      const uint4 vg = ldg_stream(wg + c), vu = ldg_stream(wu + c);
+      for (int c = part * per + lane; c < (part + 1) * per; c += 32) {
+        const uint4 vg = ldg_stream(wg + c), vu = ldg_stream(wu + c);
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        if (t < T) {
-          const uint4 xv = xs[t * n8 + c];
-          g[t] = dot8(vg, xv, g[t]);
-          u[t] = dot8(vu, xv, u[t]);
+        for (int t = 0; t < NT; ++t) {
+          if (t < T) {
+            const uint4 xv = xs[t * n8 + c];
+            g[t] = dot8(vg, xv, g[t]);
+            u[t] = dot8(vu, xv, u[t]);
+          }
         }
       }
     }
-    float gv = 0.f, uv = 0.f;
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       const float gs = warp_sum(g[t]), us = warp_sum(u[t]);
-      if (lane == t) {
-        gv = gs;
-        uv = us;
+      if (lane == 0) {
+        part_sum[rp][part][t][0] = gs;
+        part_sum[rp][part][t][1] = us;
       }
     }
-    if (lane < T) a.h[lane * Is + j] = __float2bfloat16_rn(silu_f32(gv) * uv);
+    __syncthreads();
+    if (threadIdx.x < kRowPairs * T) {
+      const int r = threadIdx.x / T, t = threadIdx.x % T;
+      if (j0 + r < Is) {
+        float gv = 0.f, uv = 0.f;
+#pragma unroll
+        for (int p = 0; p < kSplit; ++p) {
+          gv += part_sum[r][p][t][0];
+          uv += part_sum[r][p][t][1];
+        }
+        a.h[t * Is + j0 + r] = __float2bfloat16_rn(silu_f32(gv) * uv);
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -160,7 +182,7 @@ int launch_gemv_pair(const SharedArgs &a, cudaStream_t s) {
   const int rd = resident_blocks(shared_gemv_down<NT>, kGemvThreads, smem_dn);
   if (rg <= 0 || rd <= 0) return rg < 0 || rd < 0 ? NVFP4_ECUDA : NVFP4_ESHAPE;
   const int wpc = kGemvThreads / 32;
-  const int64_t gg = min64(ceil_div(a.Is, wpc), (int64_t)sms * rg);
+  const int64_t gg = min64(ceil_div(a.Is, wpc / kSplit), (int64_t)sms * rg);
   const int64_t gd = min64(ceil_div(a.H, wpc), (int64_t)sms * rd);
   if (int st = launch_pdl(shared_gemv_gateup<NT>, dim3((unsigned)gg), dim3(kGemvThreads), smem_gu,
                           s, a))

@@ -12,7 +12,8 @@
 //
 // Data flow (one stream, each kernel launched with programmatic dependent launch):
 //   route, n-tiles of 128 slots           -> routing tables
-//   quantize the x rows into padded slots -> xq [P, H/2], scale atoms, g_x [P]
+//   quantize each token's x row once      -> codes, scales and g per token
+//   copy them into the padded slots        -> xq [P, H/2], scale atoms, g_x [P]
 //   GEMM gate/up + SwiGLU                 -> h [T*K, I] bf16, slot order
 //   quantize the h rows into padded slots -> hq [P, I/2], scale atoms, g_h [P]
 //   GEMM down                             -> y [T*K, H] fp32 = w * g_dn * g_h * D
@@ -144,6 +145,69 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(Tables tb, const __nv_b
       qrow[b] = codes;
       sf[atom_offset(p, b, cols)] = (uint8_t)sc;
     }
+  }
+  pdl_launch_dependents();
+}
+
+// One warp per token: x quantized once per token (a token's slots all share its x row):
+// codes [T, H/2], the scale bytes row-major [T, H/16], the global scale g[T].
+__global__ void __launch_bounds__(256) quant_tokens_kernel(const __nv_bfloat16 *x, int64_t T,
+                                                           int64_t H, uint8_t *__restrict__ q,
+                                                           uint8_t *__restrict__ sc_rows,
+                                                           float *__restrict__ g_out) {
+  pdl_wait();   // x may come from the previous kernel
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+    const uint4 *row = reinterpret_cast<const uint4 *>(x + t * H);
+    uint32_t m = 0;
+    for (int64_t i = lane; i < H / 8; i += 32) {
+      const uint4 v = __ldg(row + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) m = max(m, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const float g = global_scale_from_amax(m << 16);
+    const BlockScaleConsts bc = block_scale_consts(g);
+    if (lane == 0) g_out[t] = g;
+    uint2 *qrow = reinterpret_cast<uint2 *>(q + t * (H / 2));
+    for (int64_t b = lane; b < H / 16; b += 32) {
+      uint32_t sc = 0;
+      qrow[b] = quantize_block16(__ldg(row + 2 * b), __ldg(row + 2 * b + 1), g, bc.c, bc.fast, &sc);
+      sc_rows[t * (H / 16) + b] = (uint8_t)sc;
+    }
+  }
+  pdl_launch_dependents();
+}
+
+// One warp per padded slot: the slot's token's codes, scales (four blocks = one 32-bit word,
+// the same word in both layouts) and global scale, copied into the slot; zeros for an empty
+// slot.
+__global__ void __launch_bounds__(256) gather_slots_kernel(Tables tb, int64_t H, int64_t K,
+                                                           int64_t P, const uint8_t *q_tok,
+                                                           const uint8_t *sc_tok,
+                                                           const float *g_tok,
+                                                           uint8_t *__restrict__ q,
+                                                           uint8_t *__restrict__ sf,
+                                                           float *__restrict__ g_out) {
+  pdl_wait();   // routing tables and the token codes
+  const int n_act = *tb.n_active;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < P; p += nwarps) {
+    int e = 0, j = 0;
+    if (!pad_slot(tb, n_act, p, e, j)) continue;
+    const bool valid = j < tb.counts[e];
+    const int64_t t = valid ? tb.perm[tb.offsets[e] + j] / K : 0;
+    const uint4 *src = reinterpret_cast<const uint4 *>(q_tok + t * (H / 2));
+    uint4 *dst = reinterpret_cast<uint4 *>(q + p * (H / 2));
+    for (int64_t i = lane; i < H / 32; i += 32) dst[i] = valid ? __ldcg(src + i) : make_uint4(0, 0, 0, 0);
+    const uint32_t *ssrc = reinterpret_cast<const uint32_t *>(sc_tok + t * (H / 16));
+    for (int64_t c = lane; c < H / 64; c += 32)
+      *reinterpret_cast<uint32_t *>(sf + atom_offset(p, 4 * c, H)) = valid ? __ldcg(ssrc + c) : 0u;
+    if (lane == 0) g_out[p] = valid ? __ldcg(g_tok + t) : 0.f;
   }
   pdl_launch_dependents();
 }
@@ -402,7 +466,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
 // Workspace of the W4A4 forward: the routed forward's, then the quantized activations.
 struct W4Layout {
-  size_t base, xq, xsf, gx, hq, hsf, gh, total;
+  size_t base, xq, xsf, gx, hq, hsf, gh, xq_tok, xsc_tok, gx_tok, total;
   int64_t P;   // padded slots provided for
 };
 W4Layout w4a4_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K) {
@@ -421,6 +485,9 @@ W4Layout w4a4_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K) {
   L.hq = take((size_t)(L.P * I / 2));
   L.hsf = take((size_t)(L.P * I / 16));
   L.gh = take((size_t)(L.P * 4));
+  L.xq_tok = take((size_t)(T * H / 2));
+  L.xsc_tok = take((size_t)(T * H / 16));
+  L.gx_tok = take((size_t)(T * 4));
   L.total = o;
   return L;
 }
@@ -589,7 +656,20 @@ int nvfp4::forward_w4a4(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   uint8_t *xq = reinterpret_cast<uint8_t *>(ws + W.xq), *xsf = reinterpret_cast<uint8_t *>(ws + W.xsf);
   uint8_t *hq = reinterpret_cast<uint8_t *>(ws + W.hq), *hsf = reinterpret_cast<uint8_t *>(ws + W.hsf);
   float *gx = reinterpret_cast<float *>(ws + W.gx), *gh = reinterpret_cast<float *>(ws + W.gh);
-  if (int s = launch_quant_rows(0, tb, x, H, K, W.P, xq, xsf, gx, stream)) return s;
+  {   // x: each token quantized once, then copied into its slots
+    uint8_t *q_tok = reinterpret_cast<uint8_t *>(ws + W.xq_tok);
+    uint8_t *s_tok = reinterpret_cast<uint8_t *>(ws + W.xsc_tok);
+    float *g_tok = reinterpret_cast<float *>(ws + W.gx_tok);
+    const int64_t bt = std::min<int64_t>(ceil_div(T * 32, 256), (int64_t)num_sms() * 8);
+    if (int s = launch_pdl(quant_tokens_kernel, dim3((unsigned)bt), dim3(256), 0, stream, x, T,
+                           H, q_tok, s_tok, g_tok))
+      return s;
+    const int64_t bp = std::min<int64_t>(ceil_div(W.P * 32, 256), (int64_t)num_sms() * 8);
+    if (int s = launch_pdl(gather_slots_kernel, dim3((unsigned)bp), dim3(256), 0, stream, tb, H,
+                           K, W.P, (const uint8_t *)q_tok, (const uint8_t *)s_tok,
+                           (const float *)g_tok, xq, xsf, gx))
+      return s;
+  }
   if (int s = mark(ev, 1, stream)) return s;
 
   W4Gemm g = {};
