@@ -593,6 +593,9 @@ class Bench:
                            "bytes_per_element": "2 (bf16) + 0.5625 (codes + scales)",
                            "l2": "inputs (19.3 GB bf16) larger than L2"},
                 "roofline": res["quantize"]["roofline"],
+                "ms_per_step": res["quantize"]["ms_per_layer"],
+                "clocks": res["quantize"]["clocks"],
+                "gpu_launches": res["quantize"]["gpu_launches"],
                 **res}
 
 
