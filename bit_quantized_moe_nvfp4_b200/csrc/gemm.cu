@@ -373,11 +373,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kg >= kSA) ok = wait(&afree[sa], ((kg / kSA) - 1) & 1) && ok;
         tc_fence_after();
         uint32_t w[NW];
-        const uint32_t *src32 =
-            reinterpret_cast<const uint32_t *>(smem + kSmemP + s * kPBytes + prow * (BK / 2)) + part * NW;
+        // The packed rows arrive with the 64-byte swizzle: 16-byte chunk c of row r sits at
+        // chunk c ^ ((r >> 1) & 3), so the rows read at one column spread over the banks.
+        const unsigned char *prow_base = smem + kSmemP + s * kPBytes + prow * (BK / 2);
+        const int sw = (prow >> 1) & 3;
 #pragma unroll
         for (int i = 0; i < NW; i += 4) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(src32 + i);
+          const int chunk = (part * NW + i) / 4;
+          const uint4 v = *reinterpret_cast<const uint4 *>(prow_base + 16 * (chunk ^ sw));
           w[i] = v.x;
           w[i + 1] = v.y;
           w[i + 2] = v.z;
@@ -558,10 +561,12 @@ int launch_gemm(const MoeArgs &a, int mode, cudaStream_t s) {
   p.scales = mode == 0 ? a.s_gu : a.s_dn;
   p.gscale = mode == 0 ? a.g_gu : a.g_dn;
   CUtensorMap tw, tb;
-  // packed weights: [E * rows_per_expert, K/2] bytes, boxes of 64 rows x 32 bytes
+  // packed weights: [E * rows_per_expert, K/2] bytes, boxes of 64 rows x BK/2 bytes with the
+  // 64-byte swizzle (the dequantize warps' reads undo it)
+  static_assert(BK / 2 == 64, "the 64-byte swizzle spans exactly one packed row");
   if (make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, mode == 0 ? a.w_gu : a.w_dn,
                (uint64_t)(p.K / 2), (uint64_t)(a.E * rows_per_expert), BK / 2, 64,
-               CU_TENSOR_MAP_SWIZZLE_NONE))
+               CU_TENSOR_MAP_SWIZZLE_64B))
     return NVFP4_ECUDA;
   // activations: [T*K + pad, K] f16 (gate/up) or bf16 (down), boxes of BN rows x 64
   // elements, 128-byte swizzle
