@@ -38,6 +38,7 @@ __device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t want, uin
 // most about three tensors are in flight: a gate/up tensor of the layer is 50 MB, and the
 // quantize pass finds it in L2 right after the amax pass brought it in.  Each input byte
 // crosses HBM once.
+constexpr int kDeqUnits = 4;   // 8-element units per dequantize thread per pass
 constexpr int kAmaxWarps = 2;
 constexpr int kAmaxThreads = 32 * kAmaxWarps;
 constexpr int kQuantThreads = 256 - kAmaxThreads;
@@ -173,38 +174,50 @@ __global__ void __launch_bounds__(256) quantize_kernel(
 // One thread per 32 elements: 16 packed bytes + 2 scale codes -> 64 bytes of bf16.
 __global__ void __launch_bounds__(256) dequantize_kernel(
     const uint8_t *__restrict__ packed, const uint8_t *__restrict__ scales,
-    const float *__restrict__ global_scale, int64_t per_tensor, int64_t n_chunks,
+    const float *__restrict__ global_scale, int64_t per_tensor, int64_t n_units,
     __nv_bfloat16 *__restrict__ out) {
+  // A unit is 8 consecutive elements: 4 packed bytes in, one 16-byte store out, so a warp's
+  // loads and stores are each one contiguous run.  kDeqUnits units per thread are loaded
+  // before any is converted.
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < n_chunks; c += stride) {
-    const int64_t e0 = c * 32;
-    const int t = (int)(e0 / per_tensor);
-    const float g = __ldg(global_scale + t);
-    const uint4 q = ldg_stream(packed + c * 16);
-    const uint32_t sc2 = __ldg(reinterpret_cast<const unsigned short *>(scales) + c);
-    const uint32_t s16 = e4m3x2_to_f16x2(sc2);          // two block scales as f16
-    const uint32_t s_lo = __byte_perm(s16, 0, 0x1010);   // (s0, s0)
-    const uint32_t s_hi = __byte_perm(s16, 0, 0x3232);   // (s1, s1)
-    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-    uint32_t o[16];
+  // tensor of element e: a double-precision estimate of e / per_tensor, corrected by one
+  const double inv_per = 1.0 / (double)per_tensor;
+  auto tensor_of = [&](int64_t e) -> int64_t {
+    int64_t t = (int64_t)((double)e * inv_per);
+    if (t * per_tensor > e) --t;
+    else if ((t + 1) * per_tensor <= e) ++t;
+    return t;
+  };
+  for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < n_units;
+       u0 += stride * kDeqUnits) {
+    uint32_t q[kDeqUnits], sc[kDeqUnits];
+    float g[kDeqUnits];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint32_t h[4];
-      e2m1x8_to_f16x2x4(words[w], h);
-      const uint32_t s = (w < 2) ? s_lo : s_hi;
+    for (int k = 0; k < kDeqUnits; ++k) {
+      const int64_t u = u0 + k * stride;
+      if (u < n_units) {
+        q[k] = __ldg(reinterpret_cast<const uint32_t *>(packed) + u);
+        sc[k] = __ldg(scales + (u >> 1));
+        g[k] = __ldg(global_scale + tensor_of(u * 8));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kDeqUnits; ++k) {
+      const int64_t u = u0 + k * stride;
+      if (u >= n_units) break;
+      const uint32_t s16 = e4m3x2_to_f16x2(sc[k] | (sc[k] << 8));   // (s, s) as f16
+      uint32_t h[4], o[4];
+      e2m1x8_to_f16x2x4(q[k], h);
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         // q * s is exact in f16 (at most 6 significant bits, within f16's range)
         __half2 qs = __hmul2(*reinterpret_cast<__half2 *>(&h[p]),
-                             *reinterpret_cast<const __half2 *>(&s));
-        uint32_t qsu = *reinterpret_cast<uint32_t *>(&qs);
-        o[w * 4 + p] = pack_bf16x2(__fmul_rn(f16_lo(qsu), g), __fmul_rn(f16_hi(qsu), g));
+                             *reinterpret_cast<const __half2 *>(&s16));
+        const uint32_t qsu = *reinterpret_cast<uint32_t *>(&qs);
+        o[p] = pack_bf16x2(__fmul_rn(f16_lo(qsu), g[k]), __fmul_rn(f16_hi(qsu), g[k]));
       }
+      stg_stream(reinterpret_cast<uint4 *>(out) + u, make_uint4(o[0], o[1], o[2], o[3]));
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(out + e0);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      stg_stream(dst + i, make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
   }
 }
 
@@ -389,14 +402,15 @@ extern "C" int nvfp4_dequantize(const uint8_t *packed, const uint8_t *scales,
   if (!packed || !scales || !global_scale || !out || n_tensors <= 0 || rows <= 0 || cols <= 0)
     return NVFP4_EINVAL;
   if (cols % 32 != 0) return NVFP4_ESHAPE;
-  // 16-byte loads of packed codes and stores of bf16, 2-byte loads of scale pairs
+  // the kernel stores bf16 in 16-byte pieces; packed and scales keep the alignment the header
+  // states (16 and 2 bytes)
   if ((reinterpret_cast<uintptr_t>(packed) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
       (reinterpret_cast<uintptr_t>(scales) & 1))
     return NVFP4_EINVAL;
   const int64_t per = rows * cols;
-  const int64_t n_chunks = n_tensors * per / 32;
-  dequantize_kernel<<<grid_for(n_chunks, 256), 256, 0, stream>>>(packed, scales, global_scale,
-                                                                 per, n_chunks, out);
+  const int64_t n_units = n_tensors * per / 8;
+  dequantize_kernel<<<grid_for(ceil_div(n_units, kDeqUnits), 256), 256, 0, stream>>>(
+      packed, scales, global_scale, per, n_units, out);
   return check_launch();
 }
 
