@@ -47,20 +47,65 @@ __device__ __forceinline__ uint32_t block_scale_code(float amax_b, float g, floa
 
 // One 16-element block (two 16-byte words of bf16: element 2k in the low half of word k)
 // -> 8 bytes of codes (element 2j in the low nibble of byte j) and its scale code.
+// Four E2M1 code pairs (8 codes, element 2j in the low nibble of byte j) of the values
+// q[0..7] as one 32-bit word: the hardware convert of each pair, the four bytes packed by one
+// move.
+__device__ __forceinline__ uint32_t e2m1x8_rn_sat(const float (&q)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+  return r;
+}
+
+// The codes of 8 elements (four bf16 pairs w[0..3]) for divisor d with r = RN(1/d): the
+// interval test of e2m1_pair_code made for four pairs at once (the lower and the upper ends
+// converted and compared as whole words); a word that differs is decided pair by pair.
+__device__ __forceinline__ uint32_t e2m1_codes8(const uint32_t *w, float d, float r) {
+  constexpr float kBelow = 1.0f - 0x1p-21f, kAbove = 1.0f + 0x1p-21f;
+  float lo[8], hi[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 q = __fmul2_rn(make_float2(bf16_lo(w[k]), bf16_hi(w[k])), make_float2(r, r));
+    const float2 a = __fmul2_rn(q, make_float2(kBelow, kBelow));
+    const float2 b = __fmul2_rn(q, make_float2(kAbove, kAbove));
+    lo[2 * k] = a.x;
+    lo[2 * k + 1] = a.y;
+    hi[2 * k] = b.x;
+    hi[2 * k + 1] = b.y;
+  }
+  const uint32_t A = e2m1x8_rn_sat(lo), B = e2m1x8_rn_sat(hi);
+  if (A == B) return A;
+  uint32_t out = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    out |= e2m1_pair_code(bf16_lo(w[k]), bf16_hi(w[k]), d, r) << (8 * k);
+  return out;
+}
+
 __device__ __forceinline__ uint2 quantize_block16(const uint4 &v0, const uint4 &v1, float g,
                                                   float c, bool fast, uint32_t *sc_out) {
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-  uint32_t m = 0;   // max of |bf16| bit patterns (same order as the values)
+  // max of |bf16| bit patterns (same order as the values), two halves at a time
+  uint32_t m2 = 0;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) m = max(m, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t a = w[k] & 0x7FFF7FFFu;
+    asm("max.u16x2 %0, %0, %1;" : "+r"(m2) : "r"(a));
+  }
+  const uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
   const uint32_t sc = block_scale_code(__uint_as_float(m << 16), g, c, fast);
   const float d = __fmul_rn(e4m3_to_f32(sc), g);
   uint32_t out[2] = {0u, 0u};
   if (d >= 0x1p-100f) {
     const float r = __frcp_rn(d);
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      out[k >> 2] |= e2m1_pair_code(bf16_lo(w[k]), bf16_hi(w[k]), d, r) << (8 * (k & 3));
+    out[0] = e2m1_codes8(w, d, r);
+    out[1] = e2m1_codes8(w + 4, d, r);
   } else if (d != 0.0f) {
 #pragma unroll
     for (int k = 0; k < 8; ++k)
