@@ -213,10 +213,11 @@ __global__ void __launch_bounds__(256) gather_slots_kernel(Tables tb, int64_t H,
 }
 
 // ------------------------------------------------------------------ the block-scaled GEMM
-constexpr int QS = 5;                            // pipeline stages (256 elements of K each)
-constexpr uint32_t kQA = 128 * 128;              // weight tile: 128 rows x 128 bytes
-constexpr uint32_t kQB = kPadN * 128;            // activation tile: 128 slots x 128 bytes
-constexpr uint32_t kQSF = 4 * 512;               // four scale atoms (256 elements of K)
+constexpr int QS = 3;                            // pipeline stages (512 elements of K each)
+constexpr uint32_t kQSub = 128 * 128;            // a 128-row tile 128 bytes (256 E2M1) wide
+constexpr uint32_t kQA = 2 * kQSub;              // weight tile: 128 rows, two K halves
+constexpr uint32_t kQB = 2 * kQSub;              // activation tile: 128 slots, two K halves
+constexpr uint32_t kQSF = 8 * 512;               // eight scale atoms (512 elements of K)
 constexpr uint32_t kQStage = kQA + kQB + 2 * kQSF;
 // Epilogue scratch: the 16-slot chunk staged for coalesced stores (down: 16 x 132 fp32;
 // gate/up: the exchanged gate and up halves, 2 x 64 x 9 fp32, then 16 x 64 bf16 of h), and
@@ -228,11 +229,11 @@ constexpr uint32_t kQBars = kQCol + kPadN * 4;
 constexpr uint32_t kQMisc = kQBars + 8 * (2 * QS + 4);
 constexpr uint32_t kQSmem = kQMisc + 16 + 1024;  // + alignment slack
 constexpr int kQThreads = 192;                   // producer, MMA, 4 epilogue warps
-// TMEM: two accumulators of 128 columns, then two buffers each of 16 columns of weight
-// scales and 16 of activation scales (four atoms of four columns).
-constexpr uint32_t kTmemSFA = 2 * kPadN, kTmemSFB = kTmemSFA + 32, kQTmemCols = 512;
+// TMEM: two accumulators of 128 columns, then two buffers each of 32 columns of weight
+// scales and 32 of activation scales (eight atoms of four columns).
+constexpr uint32_t kTmemSFA = 2 * kPadN, kTmemSFB = kTmemSFA + 64, kQTmemCols = 512;
 static_assert(kQSmem <= 227 * 1024, "shared memory budget");
-static_assert(kQStage % 1024 == 0 && kQA % 1024 == 0, "swizzled tiles on 1024-byte boundaries");
+static_assert(kQStage % 1024 == 0 && kQSub % 1024 == 0, "swizzled tiles on 1024-byte boundaries");
 
 struct W4Gemm {
   Tables tb;
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   pdl_wait();   // routing tables, quantized activations and their scales
   const int n_act = *p.tb.n_active;
   const int total = n_act > 0 ? p.tb.tile_prefix[n_act] * p.m_tiles : 0;
-  const int kblocks = p.Kred / 256;
+  const int kblocks = (p.Kred + 511) / 512;   // the last may hold one 256-element half
   const int64_t H = p.H, I = p.I;
 
   auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
@@ -322,17 +323,22 @@ __global__ void __launch_bounds__(kQThreads, 1)
           const int s = kg % QS;
           if (kg >= QS && !wait(&freeb[s], ((kg / QS) - 1) & 1)) break;
           if (*(volatile int *)abort) break;
-          mbar_arrive_expect_tx(&full[s], kQStage);
+          const int nh = min(2, (p.Kred - kb * 512) / 256);   // K halves in this stage
+          mbar_arrive_expect_tx(&full[s], (uint32_t)nh * (2 * kQSub + kQSF));
           unsigned char *A = smem + s * kQStage;
-          if (p.mode == 0) {   // 64 gate rows, then the matching 64 up rows
-            tma_load_2d(A, &tmap_w, kb * 128, (int)(e * 2 * I + mt * 64), &full[s]);
-            tma_load_2d(A + kQA / 2, &tmap_w, kb * 128, (int)(e * 2 * I + I + mt * 64), &full[s]);
-          } else {
-            tma_load_2d(A, &tmap_w, kb * 128, (int)(e * H + mt * 128), &full[s]);
+          for (int h = 0; h < nh; ++h) {
+            const int x = kb * 256 + h * 128;   // byte column of the half
+            unsigned char *Ah = A + h * kQSub;
+            if (p.mode == 0) {   // 64 gate rows, then the matching 64 up rows
+              tma_load_2d(Ah, &tmap_w, x, (int)(e * 2 * I + mt * 64), &full[s]);
+              tma_load_2d(Ah + kQSub / 2, &tmap_w, x, (int)(e * 2 * I + I + mt * 64), &full[s]);
+            } else {
+              tma_load_2d(Ah, &tmap_w, x, (int)(e * H + mt * 128), &full[s]);
+            }
+            tma_load_2d(A + kQA + h * kQSub, &tmap_x, x, (int)pad0, &full[s]);
           }
-          tma_load_2d(A + kQA, &tmap_x, kb * 128, (int)pad0, &full[s]);
-          bulk_g2s(A + kQA + kQB, sfw + kb * kQSF, kQSF, &full[s]);
-          bulk_g2s(A + kQA + kQB + kQSF, sfx + kb * kQSF, kQSF, &full[s]);
+          bulk_g2s(A + kQA + kQB, sfw + kb * kQSF, nh * (kQSF / 2), &full[s]);
+          bulk_g2s(A + kQA + kQB + kQSF, sfx + kb * kQSF, nh * (kQSF / 2), &full[s]);
         }
         if (*(volatile int *)abort) break;
       }
@@ -356,19 +362,26 @@ __global__ void __launch_bounds__(kQThreads, 1)
           const bool ok = wait(&full[s], (kg / QS) & 1);
           tc_fence_after();
           if (ok) {
+            const int nk = 4 * min(2, (p.Kred - kb * 512) / 256);   // MMAs of K = 64
             const uint32_t st = smem_u32(smem + s * kQStage);
-            const uint32_t sfa = tmem_base + kTmemSFA + 16 * (kg & 1);
-            const uint32_t sfb = tmem_base + kTmemSFB + 16 * (kg & 1);
+            const uint32_t sfa = tmem_base + kTmemSFA + 32 * (kg & 1);
+            const uint32_t sfb = tmem_base + kTmemSFB + 32 * (kg & 1);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              tmem_cp_32x128b_x4(sfa + 4 * i, smem_desc_rows16(st + kQA + kQB + 512 * i));
-              tmem_cp_32x128b_x4(sfb + 4 * i, smem_desc_rows16(st + kQA + kQB + kQSF + 512 * i));
-            }
-            const uint64_t da = smem_desc_sw128(st), db = smem_desc_sw128(st + kQA);
+            for (int i = 0; i < 8; ++i)
+              if (i < nk) {
+                tmem_cp_32x128b_x4(sfa + 4 * i, smem_desc_rows16(st + kQA + kQB + 512 * i));
+                tmem_cp_32x128b_x4(sfb + 4 * i,
+                                   smem_desc_rows16(st + kQA + kQB + kQSF + 512 * i));
+              }
 #pragma unroll
-            for (int i = 0; i < 4; ++i)   // K = 64 E2M1 = 32 bytes along the 128-byte rows
-              umma_nvfp4(d_tmem, da + 2 * i, db + 2 * i, idesc, sfa + 4 * i, sfb + 4 * i,
-                         kb > 0 || i > 0);
+            for (int i = 0; i < 8; ++i)   // K = 64 E2M1 = 32 bytes along a 128-byte row
+              if (i < nk) {
+                const uint32_t half = (uint32_t)(i / 4) * kQSub;
+                const uint64_t da = smem_desc_sw128(st + half);
+                const uint64_t db = smem_desc_sw128(st + kQA + half);
+                umma_nvfp4(d_tmem, da + 2 * (i % 4), db + 2 * (i % 4), idesc, sfa + 4 * i,
+                           sfb + 4 * i, kb > 0 || i > 0);
+              }
           }
           umma_commit(&freeb[s]);
         }
