@@ -56,6 +56,7 @@ WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int
   L.xscale = take(4 * TK);
   L.rids = take(4 * TK);   // router decisions when the call starts from logits
   L.rw = take(4 * TK);
+  L.route_blk = take(4 * (size_t)route_scratch_ints(T * K, (int)E));   // many-CTA route
   L.total = o;
   return L;
 }
@@ -226,7 +227,8 @@ static int forward_impl(const __nv_bfloat16 *x, const Routing &rt, int64_t T, in
   r.n_active = a.n_active;
   r.tile_prefix = a.tile_prefix;
   r.tile_n = gemm_tile_n();
-  if (int s = launch_route(r, stream, true)) return s;
+  if (int s = launch_route(r, stream, true, reinterpret_cast<int32_t *>(ws + L.route_blk)))
+    return s;
   if (int s = record(ev, 1, stream)) return s;
   if (int s = launch_gemm_gateup(a, stream)) return s;
   if (int s = record(ev, 2, stream)) return s;

@@ -42,7 +42,7 @@ struct MoeArgs {
 // Workspace carve-up (byte offsets, each 256-aligned).
 struct WorkspaceLayout {
   size_t flag, work, n_active, counts, offsets, active, tile_prefix, perm, inv, h, y, xs, xscale,
-      rids, rw, total;
+      rids, rw, route_blk, total;
 };
 WorkspaceLayout workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t K);
 constexpr int kGatherPadRows = 256;

@@ -39,6 +39,11 @@ struct RouteArgs {
 };
 
 size_t route_smem_bytes(int E);
-int launch_route(const RouteArgs &a, cudaStream_t stream, bool pdl);
+// Pairs per chunk of the many-CTA route; scratch ints it needs (route_scratch_ints).
+constexpr int64_t kRouteChunk = 2048;
+int64_t route_scratch_ints(int64_t n_pairs, int E);
+// The route step: one CTA, or, with scratch of route_scratch_ints(n_pairs, E) int32 and more
+// than kRouteChunk pairs, three kernels over many CTAs (the same result).
+int launch_route(const RouteArgs &a, cudaStream_t stream, bool pdl, int32_t *scratch = nullptr);
 
 }  // namespace nvfp4

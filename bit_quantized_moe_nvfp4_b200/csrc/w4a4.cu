@@ -663,7 +663,8 @@ int nvfp4::forward_w4a4(const __nv_bfloat16 *x, const int32_t *topk_ids, const f
   r.tile_prefix = a.tile_prefix;
   r.tile_n = kPadN;
   if (int s = mark(ev, 0, stream)) return s;
-  if (int s = launch_route(r, stream, true)) return s;
+  if (int s = launch_route(r, stream, true, reinterpret_cast<int32_t *>(ws + L.route_blk)))
+    return s;
 
   const Tables tb = {a.counts, a.offsets, a.active, a.n_active, a.tile_prefix, a.perm};
   uint8_t *xq = reinterpret_cast<uint8_t *>(ws + W.xq), *xsf = reinterpret_cast<uint8_t *>(ws + W.xsf);
