@@ -220,6 +220,56 @@ def test_router_argument_checks_run_before_cuda(lib):
     assert call(ws_bytes=16) == -3
 
 
+def test_shared_expert_and_layer_argument_checks_run_before_cuda(lib):
+    P, I64, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    wss = lib.moe_nvfp4_shared_workspace_size
+    wss.restype, wss.argtypes = SZ, [I64, I64]
+    assert wss(4, 2048) == 4 * 2048 * 2           # h, bf16 (a multiple of 256 already)
+    assert wss(1, 64) == 256                       # rounded up to 256 bytes
+    assert wss(0, 2048) == 0 and wss(4, 0) == 0
+    sh = lib.moe_nvfp4_shared_expert
+    sh.restype = ctypes.c_int
+    sh.argtypes = [P, I64, I64, I64, P, P, P, P, P, SZ, P]
+
+    def shared(x=fake, T=4, H=6144, Is=2048, routed=None, out=fake, ws=fake, ws_bytes=1 << 30):
+        return sh(x, T, H, Is, fake, fake, routed, out, ws, ws_bytes, None)
+
+    assert shared(x=None) == -1
+    assert shared(out=None) == -1
+    assert shared(T=0) == -1
+    assert shared(H=6100) == -2                    # not a multiple of 64
+    assert shared(Is=2000) == -2
+    assert shared(H=65536 + 64) == -2
+    assert shared(x=odd) == -1                     # 16-byte alignment
+    assert shared(routed=ctypes.c_void_p((1 << 20) + 2)) == -1   # fp32 partial: 4 bytes
+    assert shared(ws=None) == -3
+    assert shared(ws_bytes=wss(4, 2048) - 1) == -3
+    lws = lib.moe_nvfp4_layer_workspace_size
+    lws.restype, lws.argtypes = SZ, [I64, I64, I64, I64, I64, I64]
+    routed = lib.moe_nvfp4_workspace_size
+    routed.restype, routed.argtypes = SZ, [I64, I64, I64, I64, I64]
+    # routed workspace + the fp32 partial [T, H] + the shared expert's h
+    assert lws(4, 6144, 2048, 256, 8, 2048) == \
+        routed(4, 6144, 2048, 256, 8) + 4 * 6144 * 4 + wss(4, 2048)
+    assert lws(4, 6144, 2048, 256, 8, 0) == 0
+    lay = lib.moe_nvfp4_layer
+    lay.restype = ctypes.c_int
+    lay.argtypes = [P, P, I64, I64, I64, I64, I64, P, P, P, P, P, P, P, P, I64, P, P, P, P, SZ,
+                    ctypes.c_int, P]
+
+    def layer(logits=fake, ws_bytes=1 << 40, **over):
+        d = dict(dict(T=4, H=6144, I=2048, E=256, K=8, Is=2048), **over)
+        return lay(fake, logits, d["T"], d["H"], d["I"], d["E"], d["K"], fake, fake, fake, fake,
+                   fake, fake, fake, fake, d["Is"], fake, None, None, fake, ws_bytes, 0, None)
+
+    assert layer(logits=None) == -1
+    assert layer(Is=100) == -2
+    assert layer(E=4, K=8) == -2                   # the router needs K <= E
+    assert layer(ws_bytes=16) == -3
+
+
 def test_w4a4_argument_checks_run_before_cuda(lib):
     P, I64 = ctypes.c_void_p, ctypes.c_int64
     fake = ctypes.c_void_p(1 << 20)
