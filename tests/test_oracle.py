@@ -262,6 +262,39 @@ def test_moe_single_expert_is_swiglu_mlp():
         np.testing.assert_allclose(out64[t], want, rtol=1e-10, atol=1e-14)
 
 
+def test_hand_worked_moe_layer():
+    """Two constant-weight experts whose NVFP4 values are exact, so the layer output follows
+    by hand (tests/golden/hand_moe_layer.json gives the working): SwiGLU on gate rows then up
+    rows, the bf16 rounding of h, the down projection and the weighted top-k sum."""
+    with open(os.path.join(GOLDEN, "hand_moe_layer.json")) as f:
+        gd_ = json.load(f)
+    E, H, I, T = gd_["E"], gd_["H"], gd_["I"], gd_["T"]
+    gu = torch.zeros((E, 2 * I, H), dtype=torch.bfloat16)
+    dn = torch.zeros((E, H, I), dtype=torch.bfloat16)
+    for e in range(E):
+        gu[e, :I] = gd_["w_gu_gate"][e]
+        gu[e, I:] = gd_["w_gu_up"][e]
+        dn[e] = gd_["w_dn"][e]
+    x = torch.zeros((T, H), dtype=torch.bfloat16)
+    for t in range(T):
+        x[t, :2] = torch.tensor(gd_["x"][t])
+    ids = torch.tensor(gd_["ids"], dtype=torch.int32)
+    w = torch.tensor(gd_["w"], dtype=torch.float32)
+    pg, sg, gg = oracle.quantize(gu)
+    pd, sd, gdn = oracle.quantize(dn)
+    code = gd_["element_code"]
+    for e in range(E):
+        assert np.all(sg[e][:I] == gd_["gate_scale_codes"][e])
+        assert np.all(sg[e][I:] == gd_["up_scale_codes"][e])
+        assert np.all(sd[e] == gd_["down_scale_codes"][e])
+        assert np.all(pg[e] == code | (code << 4)) and np.all(pd[e] == code | (code << 4))
+    out, out64, bad = oracle.moe_forward(x, ids, w, pg, sg, gg, pd, sd, gdn)
+    assert bad == 0
+    want = np.repeat(np.asarray(gd_["out"], np.float64)[:, None], H, axis=1)
+    np.testing.assert_allclose(out64, want, rtol=1e-6, atol=0)   # fp32 g: relative 2^-24
+    assert np.array_equal(oracle.bf16_bits_to_f32(out).astype(np.float64), want)
+
+
 def test_moe_special_cases():
     H, I, E, K, T = 64, 32, 4, 2, 5
     pg, sg, gg, pd, sd, gd = _tiny_layer(9, E, H, I)
