@@ -288,11 +288,14 @@ def test_hand_worked_moe_layer():
         assert np.all(sg[e][I:] == gd_["up_scale_codes"][e])
         assert np.all(sd[e] == gd_["down_scale_codes"][e])
         assert np.all(pg[e] == code | (code << 4)) and np.all(pd[e] == code | (code << 4))
-    out, out64, bad = oracle.moe_forward(x, ids, w, pg, sg, gg, pd, sd, gdn)
-    assert bad == 0
     want = np.repeat(np.asarray(gd_["out"], np.float64)[:, None], H, axis=1)
-    np.testing.assert_allclose(out64, want, rtol=1e-6, atol=0)   # fp32 g: relative 2^-24
-    assert np.array_equal(oracle.bf16_bits_to_f32(out).astype(np.float64), want)
+    # W4A4 too: x rows (e_0; 2 e_0 - e_1) and the constant h rows quantize exactly to NVFP4
+    # (every nonzero element is its block maximum or half of it: codes 7 and 13, scale 448)
+    for w4a4 in (False, True):
+        out, out64, bad = oracle.moe_forward(x, ids, w, pg, sg, gg, pd, sd, gdn, w4a4=w4a4)
+        assert bad == 0
+        np.testing.assert_allclose(out64, want, rtol=1e-6, atol=0)   # fp32 g: 2^-24
+        assert np.array_equal(oracle.bf16_bits_to_f32(out).astype(np.float64), want)
 
 
 def test_moe_special_cases():
